@@ -1,0 +1,503 @@
+#!/usr/bin/env python
+"""Benchmark of the virtual-rank all-reduce on one B200 (or N independent replicas).
+
+One step = one all-reduce call (VRAR_ALGO_AUTO: the per-size selector plus the
+kernel it picks) over one batch of synthetic input: P = 8 virtual ranks, a
+decode-shaped message of 64 tokens x hidden 8192 bf16 (1 MiB per rank),
+values N(0, 1), seed 0.
+
+Timing: W warm-up steps, then EXACTLY K steps captured as one CUDA graph and
+replayed once between CUDA events on the launching stream, bracketed by a
+barrier and a device synchronise. Consecutive steps rotate through buffer sets
+whose total is more than 3x the L2 size, so every step reads its inputs from
+HBM. busbw = algbw * 2(P-1)/P with algbw = n * bytes-per-element / t (the
+nccl-tests convention). The roofline fraction uses the algorithm-independent
+minimum traffic B_min = 2 * P * n * s (every input read once, every output
+written once) against the measured HBM copy bandwidth.
+
+Other keys: e2e (same metric with the inputs copied from pinned host memory
+and the outputs copied back inside the timed region), cpu_baseline (the CPU
+oracle on this host), per_algo (each algorithm on the step's workload) and
+sweep (the other workload shapes and sizes).
+
+--impl reference times the CPU oracle instead (the only reference that exists
+for this method), on bounded samples of the same workload.
+
+Multi-GPU: replicas only. Each rank runs the same single-GPU workload on its
+own device; the time is the maximum over ranks and value sums all ranks' work.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "all-reduce busbw GB/s & % of HBM roofline vs size, P virtual ranks, 1 B200"
+UNIT = "GB/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD = dict(name="decode 64x8192 bf16, P=8 virtual ranks (1 MiB per rank), N(0,1), seed 0",
+                P=8, n=64 * 8192, dtype="bf16", dist="normal:0,1", seed=0)
+
+SWEEP = (
+    [dict(name=f"P=8 sweep {b >> 10} KiB per rank, N(0,1)", P=8, n=b // 2, dtype="bf16", dist="normal:0,1",
+          algos=("oneshot", "twostage", "twostage_write", "rd", "auto")) for b in
+     (128 << 10, 256 << 10, 512 << 10, 1 << 20, 2 << 20)]
+    + [dict(name="P=2 ints 128 KiB per rank", P=2, n=65536, dtype="bf16", dist="int8",
+            algos=("oneshot", "rd", "auto"))]
+    + [dict(name=f"P=32 hier 4x8 {b >> 10} KiB per rank, uniform(-1,1)", P=32, n=b // 2, dtype="bf16",
+            dist="uniform:-1,1", L=8, algos=("hier", "oneshot", "twostage_write", "auto")) for b in
+       (256 << 10, 2 << 20)]
+    + [dict(name="P=8 prefill 16384x7168 bf16 (224 MiB per rank), N(0,0.02)", P=8, n=16384 * 7168,
+            dtype="bf16", dist="normal:0,0.02", algos=("twostage", "twostage_write", "auto"), steps=20)]
+)
+
+# The oracle algorithm the reference arm times: the same summation the GPU
+# path's choice for the workload computes (the three custom all-reduce variants
+# share one order, so any of them gives the same bits).
+REFERENCE_ALGO = "twostage_write"
+
+TDT = {"bf16": torch.bfloat16, "fp32": torch.float32}
+ESZ = {"bf16": 2, "fp32": 4}
+
+
+# ---- small helpers (host logic; tested on the CPU) ---------------------------------------------
+
+def busbw_gbs(P: int, n: int, esz: int, seconds: float) -> float:
+    """nccl-tests bus bandwidth of one all-reduce of n elements per rank."""
+    if seconds <= 0:
+        return float("nan")
+    return n * esz / seconds * (2.0 * (P - 1) / P if P > 1 else 1.0) / 1e9
+
+
+def b_min_bytes(P: int, n: int, esz: int) -> int:
+    """Minimum HBM traffic of one all-reduce: every input read once, every output written once."""
+    return 2 * P * n * esz
+
+
+def rotation_sets(set_bytes: int, l2_bytes: int = L2_BYTES, cap: int = 64) -> int:
+    """Buffer sets to rotate through so that the total exceeds 3x the L2 size."""
+    return max(1, min(cap, math.ceil(3 * l2_bytes / max(1, set_bytes))))
+
+
+def load_peaks(path: str = os.path.join(ROOT, "MEASURED_PEAKS.json")):
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def parse_clocks_csv(text: str):
+    """Median SM clock under load, the max clock and the throttle reasons seen."""
+    rows = [r.strip() for r in text.splitlines() if r.strip() and not r.startswith("index")]
+    sm, smax, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        f = [c.strip() for c in r.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            cur = float(f[1].split()[0])
+            mx = float(f[2].split()[0])
+            pw = float(f[3].split()[0]) if f[3].split()[0] not in ("[N/A]", "N/A") else 0.0
+        except ValueError:
+            continue
+        smax.append(mx)
+        if pw > 150.0 or cur > 0.6 * mx:  # under load
+            sm.append(cur)
+        for name, val in zip(names, f[5:9]):
+            if val.lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "reasons": sorted(reasons), "samples_under_load": len(sm), "samples": len(rows)}
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index  # nvidia-smi -i target: PCI bus id or index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader",
+                 "-lms", "50"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        with open(self.file.name) as f:
+            text = f.read()
+        os.unlink(self.file.name)
+        return parse_clocks_csv(text)
+
+
+def gpu_bus_id(device, fallback):
+    """PCI bus id of a torch device in nvidia-smi's form (CUDA ordinals and
+    nvidia-smi indices need not agree)."""
+    try:
+        p = torch.cuda.get_device_properties(device)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return str(fallback)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank number over all ranks (a timing reduction, not data)."""
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index] if device is not None and device.type == "cuda" else None)
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "collective_all_reduce_virtual_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, or None when there is none or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None, None
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None, None
+    return e.get("dram_bytes_per_launch"), e.get("summary")
+
+
+# ---- GPU timing -------------------------------------------------------------------------------
+
+class Workload:
+    """Rotating device buffer sets holding the same seeded inputs."""
+
+    def __init__(self, spec, device, rotate=True):
+        import collective_all_reduce_virtual_b200 as vrar
+        self.vrar = vrar
+        self.spec = spec
+        self.P, self.n, self.dt = spec["P"], spec["n"], spec["dtype"]
+        self.esz = ESZ[self.dt]
+        dist = synth.parse_dist(spec["dist"])
+        gen_dev = device if self.n * self.P >= (1 << 24) else "cpu"
+        base = synth.make_inputs(self.P, self.n, TDT[self.dt], dist, seed=spec.get("seed", 0), device=gen_dev,
+                                 block=1 << 25)
+        self.base = [t.to(device) for t in base]
+        set_bytes = b_min_bytes(self.P, self.n, self.esz)
+        self.R = rotation_sets(set_bytes) if rotate else 1
+        self.ins = [self.base] + [[t.clone() for t in self.base] for _ in range(self.R - 1)]
+        self.outs = [[torch.empty_like(t) for t in self.base] for _ in range(self.R)]
+        self.in_arr = [vrar.ptr_array([t.data_ptr() for t in s]) for s in self.ins]
+        self.out_arr = [vrar.ptr_array([t.data_ptr() for t in s]) for s in self.outs]
+        self.lib = vrar.lib()
+        self.dtc = vrar.DTYPES[TDT[self.dt]]
+
+    def call(self, i: int, algo: str, stream_handle: int):
+        r = i % self.R
+        rc = self.lib.vrar_allreduce(self.in_arr[r], self.out_arr[r], self.P, self.n, self.dtc,
+                                     self.vrar.ALGOS[algo], stream_handle)
+        if rc != 0:
+            raise self.vrar.VrarError(rc, f"vrar_allreduce({algo})")
+
+    def graph(self, algo: str, count: int, offset: int = 0):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            h = torch.cuda.current_stream().cuda_stream
+            for i in range(count):
+                self.call(offset + i, algo, h)
+        return g
+
+    def free(self):
+        self.ins = self.outs = self.base = None
+
+
+def time_graph(g, world=1, device=None) -> float:
+    """Milliseconds of one replay, timed with events on the launching stream."""
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    e0.record(s)
+    g.replay()
+    e1.record(s)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    return e0.elapsed_time(e1)
+
+
+def measure_algo(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None):
+    wl.call(0, algo, torch.cuda.current_stream().cuda_stream)  # sizes the workspace outside capture
+    torch.cuda.synchronize()
+    gw = wl.graph(algo, warmup)
+    gt = wl.graph(algo, steps, offset=warmup)
+    gw.replay()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(time_graph(gt, world, device), world, device)
+    rc, info = wl.vrar.query_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} {info} after {algo}")
+    del gw, gt
+    return ms / steps
+
+
+def entry(wl: Workload, t_s: float, peak: float):
+    bw = busbw_gbs(wl.P, wl.n, wl.esz, t_s)
+    ach = b_min_bytes(wl.P, wl.n, wl.esz) / t_s / 1e9
+    return {"us": round(t_s * 1e6, 3), "busbw_gbs": round(bw, 1), "hbm_gbs_bmin": round(ach, 1),
+            "frac_bmin": round(ach / peak, 4)}
+
+
+def measure_e2e(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None):
+    """Inputs copied from pinned host memory, all-reduce, outputs copied back:
+    every step, inside the timed region (eager calls through the binding)."""
+    vrar = wl.vrar
+    h_in = [t.cpu().pin_memory() for t in wl.base]
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.base]
+    d_in, d_out = wl.ins[0], wl.outs[0]
+
+    def step():
+        for d, h in zip(d_in, h_in):
+            d.copy_(h, non_blocking=True)
+        vrar.all_reduce(d_in, d_out, algo=algo)
+        for h, d in zip(h_out, d_out):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    e0.record(s)
+    for _ in range(steps):
+        step()
+    e1.record(s)
+    e1.synchronize()
+    barrier(world, device)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device) / steps
+    bytes_in = sum(t.numel() * t.element_size() for t in h_in)
+    bytes_out = sum(t.numel() * t.element_size() for t in h_out)
+    return ms, bytes_in, bytes_out
+
+
+# ---- CPU oracle timing ----------------------------------------------------------------------------
+
+def oracle_samples(spec, algo: str, min_seconds: float, n_sample: int | None = None, max_calls=None):
+    """Time the CPU oracle on the workload (or a contiguous slice of n_sample
+    elements per rank); returns (seconds per full-size call, calls, sample text)."""
+    import oracle
+    P, n, dt = spec["P"], spec["n"], spec["dtype"]
+    m = n if n_sample is None else min(n, n_sample)
+    xs = synth.make_inputs(P, m, TDT[dt], synth.parse_dist(spec["dist"]), seed=spec.get("seed", 0))
+    xs = [t.view(torch.int16).numpy().view(np.uint16) if dt == "bf16" else t.numpy() for t in xs]
+    L = spec.get("L", 8)
+    oracle.allreduce(algo, xs, dt, L=L)  # builds/loads the library outside the timing
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        oracle.allreduce(algo, xs, dt, L=L)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or (max_calls and calls >= max_calls):
+            break
+    per_call = el / calls * (n / m)
+    sample = f"{calls} oracle calls of '{algo}' on {P} x {m} {dt} elements" + \
+             ("" if m == n else f" (a contiguous slice; time scaled by {n}/{m})")
+    return per_call, calls, sample
+
+
+# ---- arms -------------------------------------------------------------------------------------------
+
+def run_vrar(args):
+    import collective_all_reduce_virtual_b200 as vrar
+
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    peak, peak_src = load_peaks()
+
+    clocks = ClockSampler(gpu_bus_id(device, local)).start()
+    time.sleep(0.3)
+    wl = Workload(WORKLOAD, device)
+    algo_auto = vrar.select_algo(wl.P, wl.n, TDT[wl.dt])
+
+    # The timed steps: exactly K AUTO calls.
+    t_step_ms = measure_algo(wl, "auto", args.steps, args.warmup, world, device)
+    t_s = t_step_ms / 1e3
+
+    # e2e through the public call with host buffers.
+    e2e_ms, h2d, d2h = measure_e2e(wl, "auto", max(3, min(args.steps, 50)), args.warmup, world, device)
+
+    per_algo = {}
+    if not args.quick:
+        for algo in ("oneshot", "twostage", "twostage_write", "rd"):
+            per_algo[algo] = entry(wl, measure_algo(wl, algo, 200, 5, world, device) / 1e3, peak)
+    wl.free()
+
+    sweep = []
+    if not args.quick:
+        for spec in SWEEP:
+            if spec.get("L"):
+                vrar.set_group_size(spec["L"])
+            w = Workload(spec, device)
+            row = {"workload": spec["name"], "P": w.P, "n": w.n, "rotating_sets": w.R,
+                   "auto": vrar.select_algo(w.P, w.n, TDT[w.dt])}
+            for algo in spec["algos"]:
+                k = spec.get("steps", 200)
+                row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device) / 1e3, peak)
+            w.free()
+            torch.cuda.empty_cache()
+            vrar.set_group_size(8)
+            sweep.append(row)
+    clk = clocks.stop()
+
+    P, n, esz = WORKLOAD["P"], WORKLOAD["n"], ESZ[WORKLOAD["dtype"]]
+    value = world * busbw_gbs(P, n, esz, t_s)
+    achieved = b_min_bytes(P, n, esz) / t_s / 1e9
+    kernel = {"oneshot": "k_oneshot", "twostage": "k_twostage", "twostage_write": "k_twostage_write",
+              "rd": "k_rd", "hier": "k_hier"}[algo_auto]
+    traffic, traffic_src = profiled_traffic(kernel, "decode_p8_1mib")
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_step_ms, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD["name"], "P": P, "n": n, "algo": f"auto -> {algo_auto}",
+                   "l2": f"inputs rotate through {rotation_sets(b_min_bytes(P, n, esz))} buffer sets "
+                         f"({rotation_sets(b_min_bytes(P, n, esz)) * b_min_bytes(P, n, esz) >> 20} MiB) "
+                         f"> 3x the 126 MB L2",
+                   "timing": "K calls captured in one CUDA graph, replayed once between CUDA events",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, P virtual ranks"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_src} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6650 GB/s",
+                     "bytes_per_launch": b_min_bytes(P, n, esz), "kernel": kernel,
+                     "traffic_source": traffic_src},
+        "e2e": {"value": round(world * busbw_gbs(P, n, esz, e2e_ms / 1e3), 3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "per_algo": per_algo,
+        "sweep": sweep,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_call, calls, sample = oracle_samples(WORKLOAD, algo_auto, min_seconds=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(busbw_gbs(P, n, esz, per_call), 4), "unit": UNIT, "cores": 1,
+                                "kind": "oracle", "sample": sample}
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return line if rank == 0 else None
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    P, n, esz = WORKLOAD["P"], WORKLOAD["n"], ESZ[WORKLOAD["dtype"]]
+    algo = REFERENCE_ALGO
+    n_sample = 65536
+    import oracle
+    xs = synth.make_inputs(P, n_sample, TDT[WORKLOAD["dtype"]], synth.parse_dist(WORKLOAD["dist"]), seed=0)
+    xs = [t.view(torch.int16).numpy().view(np.uint16) for t in xs]
+    for _ in range(args.warmup):
+        oracle.allreduce(algo, xs, "bf16")
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.allreduce(algo, xs, "bf16")
+    el = time.perf_counter() - t0
+    per_full = el / args.steps * (n / n_sample)
+    v = busbw_gbs(P, n, esz, per_full)
+    sample = (f"each step: oracle '{algo}' on a {P} x {n_sample} bf16 slice of the workload; "
+              f"time scaled by {n}/{n_sample}")
+    return {"metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD["name"], "P": P, "n": n, "algo": algo},
+            "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("vrar", "reference"), default="vrar")
+    ap.add_argument("--quick", action="store_true", help="skip the per-algorithm table and the sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    line = run_reference(args) if args.impl == "reference" else run_vrar(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

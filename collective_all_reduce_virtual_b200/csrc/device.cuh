@@ -1,0 +1,397 @@
+// Device-side building blocks of the virtual-rank all-reduce (sm_100a).
+//
+// Sources (web pages; sections as printed on them):
+//  [CAR]   "fix(custom_all_reduce): use SYSTEM scope + ACQUIRE ordering for
+//          cross-device signal loads" (ROCm/aiter pull request 4786), "Root
+//          cause" and "Changes": per-block start/end signal arrays indexed by
+//          [block][rank], written by the peers and polled by the owner; the
+//          poll must be an ACQUIRE load at the scope the writers use, and data
+//          written with streaming (non-temporal) stores needs a fence before
+//          the completion flag.
+//  [NVRAR] "Understanding and Improving Communication Performance in
+//          Multi-node LLM Inference" (gist.science summary), Methodology item 3:
+//          "Fused Payloads" (data and flag in one 8-byte word) and
+//          "Sequence-Number Synchronization" (a per-call sequence number
+//          instead of a barrier).
+//
+// All virtual ranks live on one device, so every flag and payload access is
+// at .gpu scope: the same-device counterpart of the SYSTEM scope that [CAR]
+// needs across devices.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace vrar {
+
+constexpr int kMaxRanks = 32;
+constexpr int kThreads = 512;          // threads per CTA of every kernel
+constexpr int kMaxCtas = 2048;         // grid cap; sizes the signal arrays
+constexpr int kSigPhaseWords = kMaxCtas * kMaxRanks;
+constexpr int kPhases = 3;             // start, mid, end
+
+// Control words at the start of the workspace.
+enum Ctrl : int {
+  kStatus = 0,     // sticky error code (0 = none) until the host reads it
+  kEpoch = 1,      // sequence number of the last completed call
+  kDone = 2,       // CTAs of the running call that have finished
+  kFailEpoch = 3,  // sequence number of a call in which some wait gave up
+  kInfo = 4,       // 4 words: failing call, phase, rank, block
+  kCtrlWords = 16
+};
+
+enum Phase : uint32_t { kPhStart = 1, kPhMid = 2, kPhEnd = 3, kPhPayload = 4 };
+constexpr uint32_t kErrTimeout = 1;
+
+struct RankPtrs {
+  const void* in[kMaxRanks];
+  void* out[kMaxRanks];
+};
+
+// Kernel arguments, passed by value (they live in the constant bank).
+struct KArgs {
+  RankPtrs ptr;
+  int64_t n;         // elements per rank (the full vector)
+  int64_t items;     // 16-byte items per rank: ceil(n / elements-per-item)
+  int P;             // virtual ranks
+  int B;             // CTAs per rank
+  int L;             // group size (hierarchical)
+  int steps;         // recursive-doubling steps (log2 of the ranks doubled over)
+  int chunks;        // payload pieces in flight per thread and step
+  int edge_sync;     // run start/end barriers
+  uint32_t fault_mask;
+  uint64_t timeout_ns;
+  uint32_t* ctrl;
+  uint32_t* sig;     // kPhases x kSigPhaseWords flag words
+  uint64_t* ll;      // payload slots
+};
+
+// ---- PTX wrappers --------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Inputs: read-only for the whole launch, read once per CTA -> non-coherent
+// path without L1 allocation.
+__device__ __forceinline__ uint4 ld_input(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// Data another CTA of this launch wrote (read after an acquire): L2 only.
+__device__ __forceinline__ uint4 ld_peer(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_plain(void* p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Streaming store (evict-first), the CUDA counterpart of a non-temporal store.
+__device__ __forceinline__ void st_stream(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Two fused payload words; each 8-byte element is one single-copy-atomic access.
+__device__ __forceinline__ void st_payload2(uint64_t* p, uint64_t a, uint64_t b) {
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1,%2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+}
+
+__device__ __forceinline__ void ld_payload2(const uint64_t* p, uint64_t& a, uint64_t& b) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0,%1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+
+// ---- element types ----------------------------------------------------------------
+// An "item" is 16 bytes of one rank's vector: 8 bf16 or 4 fp32 elements.
+
+struct Bf16T {
+  using E = uint16_t;
+  static constexpr int VE = 8;
+  __device__ __forceinline__ static void widen(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  __device__ __forceinline__ static uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ __forceinline__ static uint4 narrow(const float (&f)[8]) {
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+  }
+  __device__ __forceinline__ static float elem_to_f(E e) { return __uint_as_float(static_cast<uint32_t>(e) << 16); }
+  __device__ __forceinline__ static E f_to_elem(float f) {
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<E*>(&h);
+  }
+};
+
+struct F32T {
+  using E = float;
+  static constexpr int VE = 4;
+  __device__ __forceinline__ static void widen(const uint4& v, float (&f)[4]) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+  __device__ __forceinline__ static uint4 narrow(const float (&f)[4]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+  }
+  __device__ __forceinline__ static float elem_to_f(E e) { return e; }
+  __device__ __forceinline__ static E f_to_elem(float f) { return f; }
+};
+
+// fp32 accumulator of one item. Every add is add.rn.f32: round to nearest
+// even, never contracted into an FMA, subnormals kept (no .ftz).
+template <class D>
+struct Acc {
+  float v[D::VE];
+  __device__ __forceinline__ void init(const uint4& x) { D::widen(x, v); }
+  __device__ __forceinline__ void add(const uint4& x) {
+    float f[D::VE];
+    D::widen(x, f);
+#pragma unroll
+    for (int i = 0; i < D::VE; ++i) v[i] = __fadd_rn(v[i], f[i]);
+  }
+  __device__ __forceinline__ uint4 round() const { return D::narrow(v); }
+};
+
+// rnd(f(a) + f(b)) element-wise: one recursive-doubling combine.
+template <class D>
+__device__ __forceinline__ uint4 add_round(const uint4& a, const uint4& b) {
+  Acc<D> acc;
+  acc.init(a);
+  acc.add(b);
+  return acc.round();
+}
+
+// ---- item I/O with a ragged tail ----------------------------------------------------
+// Item `it` of a rank vector of n elements; the last item may hold fewer than
+// VE elements. Missing elements load as zero and are never stored.
+
+template <class D>
+__device__ __forceinline__ int item_valid(int64_t it, int64_t n) {
+  const int64_t rem = n - it * D::VE;
+  return rem >= D::VE ? D::VE : static_cast<int>(rem);
+}
+
+template <class D>
+__device__ __forceinline__ uint4 load_item_input(const void* base, int64_t it, int64_t n) {
+  const typename D::E* p = static_cast<const typename D::E*>(base) + it * D::VE;
+  const int nv = item_valid<D>(it, n);
+  if (nv == D::VE) return ld_input(p);
+  union { uint4 u; typename D::E e[D::VE]; } t;
+#pragma unroll
+  for (int i = 0; i < D::VE; ++i) t.e[i] = i < nv ? p[i] : typename D::E(0);
+  return t.u;
+}
+
+template <class D>
+__device__ __forceinline__ uint4 load_item_peer(const void* base, int64_t it, int64_t n) {
+  const typename D::E* p = static_cast<const typename D::E*>(base) + it * D::VE;
+  const int nv = item_valid<D>(it, n);
+  if (nv == D::VE) return ld_peer(p);
+  union { uint4 u; typename D::E e[D::VE]; } t;
+#pragma unroll
+  for (int i = 0; i < D::VE; ++i) t.e[i] = i < nv ? static_cast<const volatile typename D::E*>(p)[i] : typename D::E(0);
+  return t.u;
+}
+
+template <class D, bool kStream>
+__device__ __forceinline__ void store_item(void* base, int64_t it, int64_t n, const uint4& v) {
+  typename D::E* p = static_cast<typename D::E*>(base) + it * D::VE;
+  const int nv = item_valid<D>(it, n);
+  if (nv == D::VE) {
+    if (kStream) st_stream(p, v); else st_plain(p, v);
+    return;
+  }
+  union { uint4 u; typename D::E e[D::VE]; } t;
+  t.u = v;
+  for (int i = 0; i < nv; ++i) p[i] = t.e[i];
+}
+
+// Ascending-rank fp32 sum of item `it` over ranks first .. first+count-1, one
+// rounding. Loads are issued eight at a time so that they overlap; the adds
+// stay in rank order.
+template <class D>
+__device__ __forceinline__ uint4 reduce_item(const RankPtrs& rp, int first, int count, int64_t it, int64_t n) {
+  Acc<D> acc;
+  for (int q0 = 0; q0 < count; q0 += 8) {
+    uint4 x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (q0 + j < count) x[j] = load_item_input<D>(rp.in[first + q0 + j], it, n);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (q0 + j < count) {
+        if (q0 + j == 0) acc.init(x[j]); else acc.add(x[j]);
+      }
+    }
+  }
+  return acc.round();
+}
+
+// ---- per-CTA protocol state ----------------------------------------------------------
+
+struct Cta {
+  int r;          // virtual rank this CTA acts for
+  int b;          // index of the CTA within its rank
+  uint32_t flag;  // this call's sequence number (never 0)
+};
+
+__device__ __forceinline__ Cta cta_begin(const KArgs& a) {
+  __shared__ uint32_t s_flag;
+  if (threadIdx.x == 0) {
+    uint32_t f = ld_relaxed(a.ctrl + kEpoch) + 1u;
+    s_flag = f == 0u ? 1u : f;  // 0 is the value of a never-written word
+  }
+  __syncthreads();
+  Cta c;
+  c.r = static_cast<int>(blockIdx.x % a.P);
+  c.b = static_cast<int>(blockIdx.x / a.P);
+  c.flag = s_flag;
+  return c;
+}
+
+// Every CTA counts itself out; the last one publishes this call's sequence
+// number for the next call (stream order makes it visible there) and resets
+// the counter. acq_rel orders each CTA's earlier read of kEpoch before its
+// count, so no CTA of this call can see the new value.
+__device__ __forceinline__ void cta_end(const KArgs& a, const Cta& c) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t old = atom_add_acq_rel(a.ctrl + kDone, 1u);
+    if (old == gridDim.x - 1) {
+      st_relaxed(a.ctrl + kDone, 0u);
+      st_relaxed(a.ctrl + kEpoch, c.flag);
+    }
+  }
+}
+
+__device__ __noinline__ void report_timeout(const KArgs& a, const Cta& c, uint32_t phase) {
+  if (atomicCAS(a.ctrl + kStatus, 0u, kErrTimeout) == 0u) {
+    a.ctrl[kInfo + 0] = c.flag;
+    a.ctrl[kInfo + 1] = phase;
+    a.ctrl[kInfo + 2] = static_cast<uint32_t>(c.r);
+    a.ctrl[kInfo + 3] = static_cast<uint32_t>(c.b);
+  }
+  st_relaxed(a.ctrl + kFailEpoch, c.flag);
+}
+
+// Poll `p` with acquire loads until it equals this call's flag. Gives up when
+// the time limit passes or another CTA of this call has given up; returns
+// false then. Equality (not >=) keeps the test valid across 32-bit wrap.
+__device__ __forceinline__ bool wait_flag(const uint32_t* p, const KArgs& a, const Cta& c, uint32_t phase) {
+  if (ld_acquire(p) == c.flag) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire(p) == c.flag) return true;
+    if ((it & 63u) == 0u) {
+      if (ld_relaxed(a.ctrl + kFailEpoch) == c.flag) return false;
+      if (globaltimer_ns() - t0 > a.timeout_ns) {
+        report_timeout(a, c, phase);
+        return false;
+      }
+    }
+  }
+}
+
+// Block barrier across ranks [CAR start_sync / end_sync]: block b of rank r
+// posts the call's flag into slot [r] of block b's signal row of every rank p,
+// then polls its own row until all P entries carry the flag. Threads 0..P-1
+// do one rank each. The CTA barrier before the post orders all of the CTA's
+// earlier stores before the release; the one after the poll extends the
+// acquire to the whole CTA. Returns false if any wait gave up.
+__device__ __forceinline__ bool block_barrier(const KArgs& a, const Cta& c, uint32_t phase) {
+  __syncthreads();
+  bool fail = false;
+  if (threadIdx.x < a.P) {
+    const int p = threadIdx.x;
+    uint32_t* sig = a.sig + static_cast<size_t>(phase - 1) * kSigPhaseWords;
+    if (!((a.fault_mask >> c.r) & 1u))
+      st_release(sig + (static_cast<size_t>(p) * a.B + c.b) * kMaxRanks + c.r, c.flag);
+    fail = !wait_flag(sig + (static_cast<size_t>(c.r) * a.B + c.b) * kMaxRanks + p, a, c, phase);
+  }
+  return __syncthreads_or(fail) == 0;
+}
+
+// ---- fused payload words [NVRAR "Fused Payloads"] ---------------------------------------
+// One item (16 data bytes) travels as four 8-byte words {low: 4 data bytes,
+// high: the call's sequence number}; a word is valid once its high half equals
+// the flag, so no separate signal is needed.
+
+__device__ __forceinline__ void send_item(uint64_t* slot, const uint4& v, uint32_t flag) {
+  const uint64_t hi = static_cast<uint64_t>(flag) << 32;
+  st_payload2(slot, hi | v.x, hi | v.y);
+  st_payload2(slot + 2, hi | v.z, hi | v.w);
+}
+
+// Returns false if the wait gave up (time limit, or another CTA gave up).
+__device__ __forceinline__ bool recv_item(const uint64_t* slot, uint4& v, const KArgs& a, const Cta& c) {
+  uint64_t w0, w1, w2, w3;
+  const uint32_t f = c.flag;
+  ld_payload2(slot, w0, w1);
+  ld_payload2(slot + 2, w2, w3);
+  uint64_t t0 = 0;
+  for (uint32_t it = 1; (w0 >> 32) != f || (w1 >> 32) != f || (w2 >> 32) != f || (w3 >> 32) != f; ++it) {
+    if ((w0 >> 32) != f || (w1 >> 32) != f) ld_payload2(slot, w0, w1);
+    if ((w2 >> 32) != f || (w3 >> 32) != f) ld_payload2(slot + 2, w2, w3);
+    if ((it & 63u) == 0u) {
+      if (t0 == 0) t0 = globaltimer_ns();
+      if (ld_relaxed(a.ctrl + kFailEpoch) == f) return false;
+      if (globaltimer_ns() - t0 > a.timeout_ns) {
+        report_timeout(a, c, kPhPayload);
+        return false;
+      }
+    }
+  }
+  v = make_uint4(static_cast<uint32_t>(w0), static_cast<uint32_t>(w1), static_cast<uint32_t>(w2),
+                 static_cast<uint32_t>(w3));
+  return true;
+}
+
+}  // namespace vrar

@@ -1,0 +1,281 @@
+// The all-reduce kernels. One launch does the work of all P virtual ranks:
+// CTA blockIdx.x acts as block b = blockIdx.x / P of rank r = blockIdx.x % P,
+// every rank has the same number B of CTAs, and the grid is sized so that all
+// CTAs are resident at once (the waits below need every peer to be running).
+//
+// Work split: within a rank, thread t of block b takes the items
+// b*T + t, b*T + t + B*T, ... of whatever range the phase covers (T =
+// kThreads). Every rank uses the same split, so a CTA only ever waits on the
+// CTAs with its own block index b in the other ranks.
+//
+// Sources: see device.cuh ([CAR] pull request 4786 for the custom all-reduce
+// one-shot / 2-stage / write mode and its start/end barriers; [NVRAR]
+// Methodology item 3 for the three-phase hierarchical algorithm, recursive
+// doubling, chunking, fused payloads and sequence numbers).
+#pragma once
+
+#include "device.cuh"
+
+namespace vrar {
+
+__device__ __forceinline__ int64_t lo_of(int64_t part, int64_t piece, int64_t total) {
+  const int64_t v = part * piece;
+  return v < total ? v : total;
+}
+
+// One-shot [CAR, the 1-stage kernel]: every rank reads all P inputs and
+// reduces the whole vector into its own output, between start and end
+// barriers. The P CTAs with the same b read the same items at about the same
+// time, so all but the first read of each line hit L2.
+template <class D>
+__global__ void __launch_bounds__(kThreads) k_oneshot(const KArgs a) {
+  const Cta c = cta_begin(a);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  bool ok = !a.edge_sync || block_barrier(a, c, kPhStart);
+  if (ok) {
+    void* out = a.ptr.out[c.r];
+    for (int64_t it = static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < a.items; it += stride)
+      store_item<D, true>(out, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
+    if (a.edge_sync) block_barrier(a, c, kPhEnd);
+  }
+  cta_end(a, c);
+}
+
+// 2-stage [CAR "cross_device_reduce_2stage"], pull mode. Stage 1: rank r
+// reduces slice r (ceil(items / P) items) over all P inputs into out[r]. Mid
+// barrier. Stage 2: rank r copies every other slice s out of out[s].
+template <class D>
+__global__ void __launch_bounds__(kThreads) k_twostage(const KArgs a) {
+  const Cta c = cta_begin(a);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
+  const int64_t piece = (a.items + a.P - 1) / a.P;
+  bool ok = !a.edge_sync || block_barrier(a, c, kPhStart);
+  if (ok) {
+    const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
+    void* own = a.ptr.out[c.r];
+    for (int64_t it = lo + t0; it < hi; it += stride)
+      store_item<D, false>(own, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
+    ok = block_barrier(a, c, kPhMid);
+  }
+  if (ok) {
+    void* own = a.ptr.out[c.r];
+    for (int64_t off = t0; off < piece; off += stride) {
+      // Up to 8 peer slices per batch so that the loads overlap; sources are
+      // staggered (r+1, r+2, ...) so the ranks do not all read one slice at once.
+      for (int j0 = 1; j0 < a.P; j0 += 8) {
+        uint4 v[8];
+        int64_t it[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int s = (c.r + j0 + j) % a.P;
+          it[j] = s * piece + off;
+          if (j0 + j < a.P && it[j] < lo_of(s + 1, piece, a.items)) v[j] = load_item_peer<D>(a.ptr.out[s], it[j], a.n);
+          else it[j] = -1;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j0 + j < a.P && it[j] >= 0) store_item<D, true>(own, it[j], a.n, v[j]);
+      }
+    }
+    if (a.edge_sync) block_barrier(a, c, kPhEnd);
+  }
+  cta_end(a, c);
+}
+
+// 2-stage write mode [CAR "cross_device_reduce_2stage_write_mode", Root cause
+// and change 3]: rank r reduces slice r and streams the result straight into
+// all P outputs; a device-scope fence then makes those stores visible before
+// the end barrier's flags.
+template <class D>
+__global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
+  const Cta c = cta_begin(a);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t piece = (a.items + a.P - 1) / a.P;
+  bool ok = !a.edge_sync || block_barrier(a, c, kPhStart);
+  if (ok) {
+    const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
+    for (int64_t it = lo + static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < hi; it += stride) {
+      const uint4 v = reduce_item<D>(a.ptr, 0, a.P, it, a.n);
+      for (int j = 0; j < a.P; ++j) {
+        const int p = (c.r + j) % a.P;
+        store_item<D, true>(a.ptr.out[p], it, a.n, v);
+      }
+    }
+    if (a.edge_sync) {
+      __threadfence();
+      block_barrier(a, c, kPhEnd);
+    }
+  }
+  cta_end(a, c);
+}
+
+// Recursive doubling with fused payload words [NVRAR phase 2, "Fused
+// Payloads", "Chunked Non-blocking Communication", "Sequence-Number
+// Synchronization"], over R = 2^steps ranks. The vector is cut into C chunks;
+// each thread holds one item of every chunk. At step s it stores all C items
+// (tagged with the call's sequence number) into the step-s receive slot of its
+// partner rank XOR 2^s without waiting, then takes the partner's items from its
+// own slot as they arrive and keeps rnd(own + partner).
+//
+// Payload slots: rank q's slot for step s is `per_rank` items of 32 bytes at
+// ll + ((q * steps + s) * per_rank) * 4 words. No slot is ever cleared: a
+// word belongs to this call only if its high half equals the call's flag.
+
+// Partner of rank r at step s. Flat RD: r XOR 2^s. Hierarchical (r = g*L + l):
+// the rank holding the same slice l in group g XOR 2^s.
+template <bool kHier>
+__device__ __forceinline__ int rd_partner(int r, int s, int L) {
+  if (!kHier) return r ^ (1 << s);
+  const int g = r / L, l = r % L;
+  return (g ^ (1 << s)) * L + l;
+}
+
+template <class D, int C, bool kHier>
+__device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 (&v)[C], const int64_t (&idx)[C],
+                                            const bool (&val)[C], int64_t per_rank) {
+  const bool mute = (a.fault_mask >> c.r) & 1u;
+  for (int s = 0; s < a.steps; ++s) {
+    const int q = rd_partner<kHier>(c.r, s, a.L);
+    uint64_t* dst = a.ll + (static_cast<size_t>(q) * a.steps + s) * per_rank * 4;
+    const uint64_t* src = a.ll + (static_cast<size_t>(c.r) * a.steps + s) * per_rank * 4;
+    if (!mute) {
+#pragma unroll
+      for (int k = 0; k < C; ++k)
+        if (val[k]) send_item(dst + idx[k] * 4, v[k], c.flag);
+    }
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      if (val[k]) {
+        uint4 w;
+        if (!recv_item(src + idx[k] * 4, w, a, c)) return false;
+        v[k] = add_round<D>(v[k], w);
+      }
+    }
+  }
+  return true;
+}
+
+template <class D, int C>
+__global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
+  const Cta c = cta_begin(a);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
+  const int64_t per_chunk = (a.items + C - 1) / C;
+  bool ok = true;
+  for (int64_t base = 0; base < per_chunk && ok; base += stride) {
+    const int64_t j = base + t0;
+    uint4 v[C];
+    int64_t idx[C];
+    bool val[C];
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      idx[k] = k * per_chunk + j;
+      val[k] = j < per_chunk && idx[k] < a.items;
+      if (val[k]) v[k] = load_item_input<D>(a.ptr.in[c.r], idx[k], a.n);
+    }
+    ok = rd_exchange<D, C, false>(a, c, v, idx, val, a.items);
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < C; ++k)
+        if (val[k]) store_item<D, true>(a.ptr.out[c.r], idx[k], a.n, v[k]);
+    }
+  }
+  cta_end(a, c);
+}
+
+// Hierarchical all-reduce [NVRAR Methodology item 3, phases 1-3] with P = G*L
+// ranks, rank r = g*L + l. Phase 1 (in-group reduce-scatter): rank (g, l)
+// reduces slice l (ceil(items / L) items) over the L ranks of group g in
+// ascending order, one rounding. Phase 2 (inter-group recursive doubling):
+// log2 G steps of fused-payload exchange with partner (g XOR 2^s, l). Phase 3
+// (in-group all-gather): rank (g, l) streams slice l into the outputs of all
+// L ranks of group g. Slices are cut into C chunks as in k_rd.
+template <class D, int C>
+__global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
+  const Cta c = cta_begin(a);
+  const int L = a.L, g = c.r / L, l = c.r % L;
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
+  const int64_t piece = (a.items + L - 1) / L;
+  const int64_t lo = lo_of(l, piece, a.items), len = lo_of(l + 1, piece, a.items) - lo;
+  const int64_t per_chunk = (len + C - 1) / C;
+  bool ok = true;
+  for (int64_t base = 0; base < per_chunk && ok; base += stride) {
+    const int64_t j = base + t0;
+    uint4 v[C];
+    int64_t idx[C];
+    bool val[C];
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      idx[k] = k * per_chunk + j;
+      val[k] = j < per_chunk && idx[k] < len;
+      if (val[k]) v[k] = reduce_item<D>(a.ptr, g * L, L, lo + idx[k], a.n);
+    }
+    ok = rd_exchange<D, C, true>(a, c, v, idx, val, piece);
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < C; ++k) {
+        if (!val[k]) continue;
+        for (int jj = 0; jj < L; ++jj) {
+          const int lp = (l + jj) % L;
+          store_item<D, true>(a.ptr.out[g * L + lp], lo + idx[k], a.n, v[k]);
+        }
+      }
+    }
+  }
+  cta_end(a, c);
+}
+
+// Standalone reduce-scatter [NVRAR phase 1 over one group]: rank p writes
+// elements [p*m, (p+1)*m) of the ascending-rank sum into out[p], m = n / P.
+// Needs no flags. 16-byte path when m is a multiple of the item size (so
+// every slice starts on a 16-byte boundary), element path otherwise.
+template <class D>
+__global__ void __launch_bounds__(kThreads) k_reduce_scatter(const KArgs a) {
+  const int r = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t t0 = static_cast<int64_t>(b) * kThreads + threadIdx.x;
+  const int64_t m = a.n / a.P;
+  if (m % D::VE == 0) {
+    const int64_t mi = m / D::VE;
+    for (int64_t j = t0; j < mi; j += stride)
+      store_item<D, true>(a.ptr.out[r], j, m, reduce_item<D>(a.ptr, 0, a.P, r * mi + j, a.n));
+  } else {
+    using E = typename D::E;
+    for (int64_t e = t0; e < m; e += stride) {
+      const int64_t src = r * m + e;
+      float acc = D::elem_to_f(static_cast<const E*>(a.ptr.in[0])[src]);
+      for (int q = 1; q < a.P; ++q) acc = __fadd_rn(acc, D::elem_to_f(static_cast<const E*>(a.ptr.in[q])[src]));
+      static_cast<E*>(a.ptr.out[r])[e] = D::f_to_elem(acc);
+    }
+  }
+}
+
+// Standalone all-gather [NVRAR phase 3 over one group], push form: rank s
+// reads its n/P elements once and streams them to offset s*m of all P outputs.
+template <class D>
+__global__ void __launch_bounds__(kThreads) k_all_gather(const KArgs a) {
+  const int s = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t t0 = static_cast<int64_t>(b) * kThreads + threadIdx.x;
+  const int64_t m = a.n / a.P;
+  if (m % D::VE == 0) {
+    const int64_t mi = m / D::VE;
+    for (int64_t j = t0; j < mi; j += stride) {
+      const uint4 v = load_item_input<D>(a.ptr.in[s], j, m);
+      for (int jj = 0; jj < a.P; ++jj) {
+        const int p = (s + jj) % a.P;
+        store_item<D, true>(a.ptr.out[p], s * mi + j, a.n, v);
+      }
+    }
+  } else {
+    using E = typename D::E;
+    for (int64_t e = t0; e < m; e += stride) {
+      const E v = static_cast<const E*>(a.ptr.in[s])[e];
+      for (int p = 0; p < a.P; ++p) static_cast<E*>(a.ptr.out[p])[s * m + e] = v;
+    }
+  }
+}
+
+}  // namespace vrar

@@ -1,0 +1,484 @@
+// Host side of the C ABI declared in include/vrar.h: argument checks, the
+// per-device workspace, grid sizing, the per-size selector and the status
+// word. Every call queues exactly one kernel on the caller's stream.
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+#include "vrar.h"
+
+namespace vrar {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct Settings {
+  std::atomic<int> group_size{8};
+  std::atomic<int> rd_chunks{4};
+  std::atomic<int> edge_sync{1};
+  std::atomic<uint64_t> timeout_ns{2000000000ull};
+  std::atomic<uint32_t> fault_mask{0};
+};
+Settings g_set;
+
+// Library-owned device memory of one device: control words, the three
+// signal arrays and the payload slots, zeroed when allocated.
+struct Workspace {
+  uint32_t* ctrl = nullptr;  // kCtrlWords words, then kPhases * kSigPhaseWords signal words
+  uint32_t* sig = nullptr;
+  uint64_t* ll = nullptr;
+  size_t ll_bytes = 0;
+  int sms = 0;
+};
+
+std::mutex g_mu;
+Workspace g_ws[kMaxDevices];
+
+size_t elem_size(vrar_dtype_t dt) { return dt == VRAR_BF16 ? 2 : 4; }
+int64_t per_item(vrar_dtype_t dt) { return dt == VRAR_BF16 ? 8 : 4; }
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int ilog2(int x) {
+  int s = 0;
+  while ((1 << s) < x) ++s;
+  return s;
+}
+
+int cuda_fail(cudaError_t e) {
+  (void)e;
+  cudaGetLastError();  // clear the non-sticky error so later calls start clean
+  return VRAR_ECUDA;
+}
+
+int current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (*dev < 0 || *dev >= kMaxDevices) return VRAR_ECUDA;
+  return VRAR_OK;
+}
+
+// Allocate (once) the control + signal block and grow the payload slots to at
+// least ll_need bytes. Growing frees the old slots after a device-wide sync.
+int ensure_workspace(int dev, size_t ll_need, Workspace** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& w = g_ws[dev];
+  if (!w.ctrl) {
+    const size_t words = kCtrlWords + static_cast<size_t>(kPhases) * kSigPhaseWords;
+    void* p = nullptr;
+    if (cudaMalloc(&p, words * sizeof(uint32_t)) != cudaSuccess) {
+      cudaGetLastError();
+      return VRAR_ENOMEM;
+    }
+    if (cudaMemset(p, 0, words * sizeof(uint32_t)) != cudaSuccess) {
+      cudaFree(p);
+      return cuda_fail(cudaErrorUnknown);
+    }
+    w.ctrl = static_cast<uint32_t*>(p);
+    w.sig = w.ctrl + kCtrlWords;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+    w.sms = sms;
+  }
+  if (ll_need > w.ll_bytes) {
+    if (w.ll) {
+      if (cudaDeviceSynchronize() != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+      cudaFree(w.ll);
+      w.ll = nullptr;
+      w.ll_bytes = 0;
+    }
+    const size_t bytes = (ll_need + (1u << 20) - 1) & ~static_cast<size_t>((1u << 20) - 1);
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return VRAR_ENOMEM;
+    }
+    if (cudaMemset(p, 0, bytes) != cudaSuccess) {
+      cudaFree(p);
+      return cuda_fail(cudaErrorUnknown);
+    }
+    w.ll = static_cast<uint64_t*>(p);
+    w.ll_bytes = bytes;
+  }
+  *out = &w;
+  return VRAR_OK;
+}
+
+// ---- argument checks -------------------------------------------------------------------
+
+struct Range {
+  uintptr_t lo, hi;
+};
+
+bool overlap(const Range& a, const Range& b) { return a.lo < b.hi && b.lo < a.hi; }
+
+int check_buffers(const void* const in[], void* const out[], int P, size_t in_elems, size_t out_elems,
+                  vrar_dtype_t dt) {
+  if (!in || !out) return VRAR_EINVAL;
+  if (P < 1 || P > kMaxRanks) return VRAR_EINVAL;
+  if (dt != VRAR_BF16 && dt != VRAR_FP32) return VRAR_EINVAL;
+  const size_t es = elem_size(dt);
+  if (in_elems > (SIZE_MAX / 2) / es || out_elems > (SIZE_MAX / 2) / es) return VRAR_EINVAL;
+  Range ri[kMaxRanks], ro[kMaxRanks];
+  for (int p = 0; p < P; ++p) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(in[p]), b = reinterpret_cast<uintptr_t>(out[p]);
+    if (!a || !b || (a & 15u) || (b & 15u)) return VRAR_EINVAL;
+    ri[p] = {a, a + in_elems * es};
+    ro[p] = {b, b + out_elems * es};
+  }
+  if (in_elems == 0 || out_elems == 0) return VRAR_OK;
+  for (int q = 0; q < P; ++q) {
+    for (int p = 0; p < P; ++p)
+      if (overlap(ro[q], ri[p])) return VRAR_EINVAL;
+    for (int p = q + 1; p < P; ++p)
+      if (overlap(ro[q], ro[p])) return VRAR_EINVAL;
+  }
+  return VRAR_OK;
+}
+
+int check_shape(vrar_algo_t algo, int P, int L) {
+  switch (algo) {
+    case VRAR_ALGO_ONESHOT:
+    case VRAR_ALGO_TWOSTAGE:
+    case VRAR_ALGO_TWOSTAGE_WRITE:
+      return VRAR_OK;
+    case VRAR_ALGO_RD:
+      return is_pow2(P) ? VRAR_OK : VRAR_ENOTSUP;
+    case VRAR_ALGO_HIER:
+      return (L >= 1 && P % L == 0 && is_pow2(P / L)) ? VRAR_OK : VRAR_ENOTSUP;
+    default:
+      return VRAR_EINVAL;
+  }
+}
+
+// Payload-slot bytes (RD / HIER): P ranks x steps x items-per-slot x 32 bytes.
+size_t ll_bytes_for(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L) {
+  const int64_t items = (static_cast<int64_t>(n) + per_item(dt) - 1) / per_item(dt);
+  if (algo == VRAR_ALGO_RD) return static_cast<size_t>(P) * ilog2(P) * items * 32;
+  if (algo == VRAR_ALGO_HIER) {
+    const int64_t piece = (items + L - 1) / L;
+    return static_cast<size_t>(P) * ilog2(P / L) * piece * 32;
+  }
+  return 0;
+}
+
+// ---- launch -----------------------------------------------------------------------------
+
+using KernelFn = void (*)(KArgs);
+
+// CTAs resident per SM for a kernel (cached per kernel and device).
+int resident_ctas(KernelFn fn, int dev, int sms) {
+  struct Entry {
+    KernelFn fn;
+    int dev;
+    int occ;
+  };
+  static std::mutex mu;
+  static Entry cache[256];
+  static int used = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == fn && cache[i].dev == dev) return cache[i].occ * sms;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, 0) != cudaSuccess || occ < 1) {
+    cudaGetLastError();
+    occ = 1;
+  }
+  if (used < 256) cache[used++] = {fn, dev, occ};
+  return occ * sms;
+}
+
+// CTAs per rank: enough for one item per thread over `work_items` (the items
+// one rank handles), at most what keeps the whole grid resident.
+int blocks_per_rank(int64_t work_items, int P, int max_ctas) {
+  const int64_t want = std::max<int64_t>(1, (work_items + kThreads - 1) / kThreads);
+  const int64_t cap = std::max(1, std::min(max_ctas, kMaxCtas) / P);
+  return static_cast<int>(std::min(want, cap));
+}
+
+template <class D>
+KernelFn pick_kernel(vrar_algo_t algo, int C) {
+#define VRAR_CHUNK_CASES(K)          \
+  switch (C) {                       \
+    case 1: return K<D, 1>;          \
+    case 2: return K<D, 2>;          \
+    case 3: return K<D, 3>;          \
+    case 4: return K<D, 4>;          \
+    case 5: return K<D, 5>;          \
+    case 6: return K<D, 6>;          \
+    case 7: return K<D, 7>;          \
+    default: return K<D, 8>;         \
+  }
+  switch (algo) {
+    case VRAR_ALGO_ONESHOT: return k_oneshot<D>;
+    case VRAR_ALGO_TWOSTAGE: return k_twostage<D>;
+    case VRAR_ALGO_TWOSTAGE_WRITE: return k_twostage_write<D>;
+    case VRAR_ALGO_RD: VRAR_CHUNK_CASES(k_rd)
+    case VRAR_ALGO_HIER: VRAR_CHUNK_CASES(k_hier)
+    default: return nullptr;
+  }
+#undef VRAR_CHUNK_CASES
+}
+
+int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream) {
+  fn<<<grid, kThreads, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? VRAR_OK : VRAR_ECUDA;
+}
+
+const char* algo_name(int a) {
+  switch (a) {
+    case VRAR_ALGO_ONESHOT: return "oneshot";
+    case VRAR_ALGO_TWOSTAGE: return "twostage";
+    case VRAR_ALGO_TWOSTAGE_WRITE: return "twostage_write";
+    case VRAR_ALGO_RD: return "rd";
+    case VRAR_ALGO_HIER: return "hier";
+    default: return "auto";
+  }
+}
+
+// VRAR_ALGO from the environment (read once): forces the AUTO choice.
+int env_algo() {
+  static int cached = -2;
+  if (cached != -2) return cached;
+  int v = -1;
+  if (const char* s = std::getenv("VRAR_ALGO")) {
+    for (int a = VRAR_ALGO_ONESHOT; a <= VRAR_ALGO_HIER; ++a)
+      if (std::strcmp(s, algo_name(a)) == 0) v = a;
+  }
+  cached = v;
+  return v;
+}
+
+int select_algo(int P, size_t n, vrar_dtype_t dt) {
+  const size_t bytes = n * elem_size(dt);
+  if (P <= 1) return VRAR_ALGO_ONESHOT;
+  if (bytes <= (256u << 10)) return VRAR_ALGO_ONESHOT;
+  return VRAR_ALGO_TWOSTAGE_WRITE;
+}
+
+}  // namespace
+}  // namespace vrar
+
+using namespace vrar;
+
+extern "C" {
+
+int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, size_t n, vrar_dtype_t dtype,
+                   vrar_algo_t algo, vrar_stream_t stream) {
+  int rc = check_buffers(rank_in, rank_out, P, n, n, dtype);
+  if (rc != VRAR_OK) return rc;
+  if (algo == VRAR_ALGO_AUTO) {
+    const int forced = env_algo();
+    algo = static_cast<vrar_algo_t>(forced > 0 ? forced : select_algo(P, n, dtype));
+  }
+  const int L = g_set.group_size.load();
+  if ((rc = check_shape(algo, P, L)) != VRAR_OK) return rc;
+  if (n == 0) return VRAR_OK;
+
+  int dev = 0;
+  if ((rc = current_device(&dev)) != VRAR_OK) return rc;
+  Workspace* ws = nullptr;
+  if ((rc = ensure_workspace(dev, ll_bytes_for(algo, P, n, dtype, L), &ws)) != VRAR_OK) return rc;
+
+  const int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
+  KernelFn fn = dtype == VRAR_BF16 ? pick_kernel<Bf16T>(algo, C) : pick_kernel<F32T>(algo, C);
+  if (!fn) return VRAR_EINVAL;
+
+  KArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int p = 0; p < P; ++p) {
+    a.ptr.in[p] = rank_in[p];
+    a.ptr.out[p] = rank_out[p];
+  }
+  a.n = static_cast<int64_t>(n);
+  a.items = (a.n + per_item(dtype) - 1) / per_item(dtype);
+  a.P = P;
+  a.L = L;
+  a.chunks = C;
+  a.edge_sync = g_set.edge_sync.load();
+  a.fault_mask = g_set.fault_mask.load();
+  a.timeout_ns = g_set.timeout_ns.load();
+  a.ctrl = ws->ctrl;
+  a.sig = ws->sig;
+  a.ll = ws->ll;
+
+  int64_t work = a.items;  // items one rank handles in its main loop
+  switch (algo) {
+    case VRAR_ALGO_ONESHOT: work = a.items; break;
+    case VRAR_ALGO_TWOSTAGE:
+    case VRAR_ALGO_TWOSTAGE_WRITE: work = (a.items + P - 1) / P; break;
+    case VRAR_ALGO_RD:
+      a.steps = ilog2(P);
+      work = (a.items + C - 1) / C;
+      break;
+    case VRAR_ALGO_HIER: {
+      a.steps = ilog2(P / L);
+      const int64_t piece = (a.items + L - 1) / L;
+      work = (piece + C - 1) / C;
+      break;
+    }
+    default: break;
+  }
+  a.B = blocks_per_rank(work, P, resident_ctas(fn, dev, ws->sms));
+  return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vrar_reduce_scatter(const void* const rank_in[], void* const rank_out[], int P, size_t n, vrar_dtype_t dtype,
+                        vrar_stream_t stream) {
+  if (P < 1 || P > kMaxRanks) return VRAR_EINVAL;
+  if (n % static_cast<size_t>(P) != 0) return VRAR_EINVAL;
+  int rc = check_buffers(rank_in, rank_out, P, n, n / P, dtype);
+  if (rc != VRAR_OK) return rc;
+  if (n == 0) return VRAR_OK;
+  int dev = 0;
+  if ((rc = current_device(&dev)) != VRAR_OK) return rc;
+  Workspace* ws = nullptr;
+  if ((rc = ensure_workspace(dev, 0, &ws)) != VRAR_OK) return rc;
+  KernelFn fn = dtype == VRAR_BF16 ? k_reduce_scatter<Bf16T> : k_reduce_scatter<F32T>;
+  KArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int p = 0; p < P; ++p) {
+    a.ptr.in[p] = rank_in[p];
+    a.ptr.out[p] = rank_out[p];
+  }
+  a.n = static_cast<int64_t>(n);
+  a.P = P;
+  const int64_t m = a.n / P;
+  const int64_t work = (m % per_item(dtype) == 0) ? m / per_item(dtype) : m;
+  a.B = blocks_per_rank(work, P, resident_ctas(fn, dev, ws->sms));
+  return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, size_t n, vrar_dtype_t dtype,
+                    vrar_stream_t stream) {
+  if (P < 1 || P > kMaxRanks) return VRAR_EINVAL;
+  if (n % static_cast<size_t>(P) != 0) return VRAR_EINVAL;
+  int rc = check_buffers(rank_in, rank_out, P, n / P, n, dtype);
+  if (rc != VRAR_OK) return rc;
+  if (n == 0) return VRAR_OK;
+  int dev = 0;
+  if ((rc = current_device(&dev)) != VRAR_OK) return rc;
+  Workspace* ws = nullptr;
+  if ((rc = ensure_workspace(dev, 0, &ws)) != VRAR_OK) return rc;
+  KernelFn fn = dtype == VRAR_BF16 ? k_all_gather<Bf16T> : k_all_gather<F32T>;
+  KArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int p = 0; p < P; ++p) {
+    a.ptr.in[p] = rank_in[p];
+    a.ptr.out[p] = rank_out[p];
+  }
+  a.n = static_cast<int64_t>(n);
+  a.P = P;
+  const int64_t m = a.n / P;
+  const int64_t work = (m % per_item(dtype) == 0) ? m / per_item(dtype) : m;
+  a.B = blocks_per_rank(work, P, resident_ctas(fn, dev, ws->sms));
+  return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype) {
+  if (P < 1 || P > kMaxRanks || (dtype != VRAR_BF16 && dtype != VRAR_FP32)) return VRAR_EINVAL;
+  return select_algo(P, n, dtype);
+}
+
+int vrar_set_group_size(int L) {
+  if (L < 1 || L > kMaxRanks) return VRAR_EINVAL;
+  g_set.group_size = L;
+  return VRAR_OK;
+}
+int vrar_get_group_size(void) { return g_set.group_size.load(); }
+
+int vrar_set_rd_chunks(int C) {
+  if (C < 1 || C > 8) return VRAR_EINVAL;
+  g_set.rd_chunks = C;
+  return VRAR_OK;
+}
+int vrar_get_rd_chunks(void) { return g_set.rd_chunks.load(); }
+
+int vrar_set_edge_sync(int on) {
+  g_set.edge_sync = on ? 1 : 0;
+  return VRAR_OK;
+}
+int vrar_get_edge_sync(void) { return g_set.edge_sync.load(); }
+
+int vrar_set_spin_timeout_ns(uint64_t ns) {
+  if (ns < 100000ull || ns > 60000000000ull) return VRAR_EINVAL;
+  g_set.timeout_ns = ns;
+  return VRAR_OK;
+}
+uint64_t vrar_get_spin_timeout_ns(void) { return g_set.timeout_ns.load(); }
+
+int vrar_query_status(vrar_stream_t stream, uint32_t info[4]) {
+  int dev = 0;
+  int rc = current_device(&dev);
+  if (rc != VRAR_OK) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& w = g_ws[dev];
+  if (info) std::memset(info, 0, 4 * sizeof(uint32_t));
+  if (!w.ctrl) return VRAR_OK;
+  uint32_t h[kCtrlWords];
+  if (cudaMemcpy(h, w.ctrl, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+  if (h[kStatus] == 0) return VRAR_OK;
+  if (info) std::memcpy(info, h + kInfo, 4 * sizeof(uint32_t));
+  const uint32_t zero[5] = {0, 0, 0, 0, 0};
+  if (cudaMemcpy(w.ctrl + kStatus, zero, sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(w.ctrl + kInfo, zero, 4 * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess)
+    return cuda_fail(cudaErrorUnknown);
+  return h[kStatus] == kErrTimeout ? VRAR_ETIMEDOUT : VRAR_ECUDA;
+}
+
+int vrar_reserve(size_t bytes) {
+  int dev = 0;
+  int rc = current_device(&dev);
+  if (rc != VRAR_OK) return rc;
+  Workspace* ws = nullptr;
+  return ensure_workspace(dev, bytes, &ws);
+}
+
+size_t vrar_workspace_bytes(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t algo) {
+  if (P < 1 || P > kMaxRanks || (dtype != VRAR_BF16 && dtype != VRAR_FP32)) return 0;
+  if (algo == VRAR_ALGO_AUTO) algo = static_cast<vrar_algo_t>(select_algo(P, n, dtype));
+  const int L = g_set.group_size.load();
+  if (check_shape(algo, P, L) != VRAR_OK) return 0;
+  return ll_bytes_for(algo, P, n, dtype, L);
+}
+
+int vrar_reset(void) {
+  int dev = 0;
+  int rc = current_device(&dev);
+  if (rc != VRAR_OK) return rc;
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& w = g_ws[dev];
+  if (cudaDeviceSynchronize() != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+  if (w.ll) cudaFree(w.ll);
+  if (w.ctrl) cudaFree(w.ctrl);
+  w = Workspace();
+  return VRAR_OK;
+}
+
+int vrar_debug_set_fault_mask(uint32_t mask) {
+  g_set.fault_mask = mask;
+  return VRAR_OK;
+}
+
+const char* vrar_strerror(int code) {
+  switch (code) {
+    case VRAR_OK: return "success";
+    case VRAR_EINVAL: return "invalid argument";
+    case VRAR_ENOTSUP: return "shape not supported by the algorithm";
+    case VRAR_ENOMEM: return "workspace allocation failed";
+    case VRAR_ECUDA: return "CUDA runtime error";
+    case VRAR_ETIMEDOUT: return "a device wait timed out";
+    default: return "unknown error";
+  }
+}
+
+int vrar_version(void) { return VRAR_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,202 @@
+/*
+ * vrar — virtual-rank all-reduce on one GPU (C ABI).
+ *
+ * P "virtual ranks" are P buffers in the memory of ONE CUDA device. A call
+ * does every rank's reduce and exchange work on that device in a single
+ * kernel launch: thread blocks act as the ranks and synchronise through flag
+ * words and sequence-numbered 8-byte payload words in device memory. There is
+ * no cross-GPU traffic and no collective library underneath.
+ *
+ * Sources for the operations (web pages; sections as printed on them):
+ *  [CAR]   "fix(custom_all_reduce): use SYSTEM scope + ACQUIRE ordering for
+ *          cross-device signal loads" (ROCm/aiter pull request 4786),
+ *          "Summary" and "Root cause": start_sync / end_sync flag barriers
+ *          polled with acquire loads, the 2-stage reduce-scatter + all-gather
+ *          kernel, and its write mode, which streams the reduced slice into
+ *          every rank's registered output and fences before end_sync.
+ *  [NVRAR] "Understanding and Improving Communication Performance in
+ *          Multi-node LLM Inference" (gist.science technical summary of
+ *          arXiv 2511.09557), "Methodology" item 3 "Proposed Solution
+ *          (NVRAR)": intra-node reduce-scatter, inter-node recursive doubling,
+ *          intra-node all-gather; chunked non-blocking communication; data and
+ *          flag fused into one 8-byte payload; sequence numbers in place of
+ *          global barriers.
+ *
+ * Conventions for every call below
+ *  - Buffers: rank_in[p] / rank_out[p] are DEVICE pointers on the CURRENT
+ *    device (cudaGetDevice), each 16-byte aligned, each the start of a
+ *    contiguous vector. The caller owns them. rank_in[] must not change, and
+ *    rank_out[] must not be read, until the stream has passed the call.
+ *  - The pointer arrays themselves are HOST arrays of P entries. They are
+ *    copied into the kernel's parameters by value, so they may be freed or
+ *    reused as soon as the call returns.
+ *  - n is the number of ELEMENTS of the full per-rank vector.
+ *  - Elements are bf16 (VRAR_BF16) or IEEE binary32 (VRAR_FP32). Sums are
+ *    formed in binary32 with round-to-nearest-even adds and rounded to the
+ *    element type with round-to-nearest-even (subnormals kept).
+ *  - Out-of-place only: no output may overlap any input or another output.
+ *  - 1 <= P <= VRAR_MAX_RANKS. n == 0 is a valid no-op.
+ *  - The call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream). It returns once the kernel is queued. Calls that run
+ *    concurrently on different streams of one device are not supported: they
+ *    share the device workspace.
+ *  - The library owns a per-device workspace (flag words, payload slots, the
+ *    sequence counter and a status word), allocated and zeroed on first use
+ *    and grown when a larger call needs more. Growing allocates, which is not
+ *    allowed while a stream is being captured into a CUDA graph: make one call
+ *    of the largest shape (or call vrar_reserve) before capturing.
+ *  - Return value: VRAR_OK, or a negative VRAR_E* code. Argument errors are
+ *    found on the host before anything is queued. A device wait that hits
+ *    its time limit cannot be returned by the call that queued it: the kernel
+ *    records VRAR_ETIMEDOUT in the status word, which vrar_query_status reads.
+ *    No C++ exception crosses this interface.
+ */
+#ifndef VRAR_H
+#define VRAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define VRAR_API __attribute__((visibility("default")))
+#else
+#define VRAR_API
+#endif
+
+#define VRAR_MAX_RANKS 32
+#define VRAR_VERSION 1
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* vrar_stream_t;
+
+typedef enum {
+    VRAR_BF16 = 0,
+    VRAR_FP32 = 1
+} vrar_dtype_t;
+
+typedef enum {
+    VRAR_ALGO_AUTO = 0,           /* per-size choice, see vrar_select_algo */
+    VRAR_ALGO_ONESHOT = 1,        /* [CAR] 1-stage: every rank reads all P inputs */
+    VRAR_ALGO_TWOSTAGE = 2,       /* [CAR] reduce-scatter, mid barrier, pull all-gather */
+    VRAR_ALGO_TWOSTAGE_WRITE = 3, /* [CAR] write mode: owner streams its slice to all P outputs */
+    VRAR_ALGO_RD = 4,             /* [NVRAR] recursive doubling with fused 8-byte payloads */
+    VRAR_ALGO_HIER = 5            /* [NVRAR] group RS -> inter-group RD -> group AG */
+} vrar_algo_t;
+
+enum {
+    VRAR_OK = 0,
+    VRAR_EINVAL = -1,    /* bad argument: null/misaligned pointer, P or n out of range, overlap */
+    VRAR_ENOTSUP = -2,   /* shape the algorithm does not define (RD: P not 2^k; HIER: L does not
+                            divide P or P/L not 2^k) */
+    VRAR_ENOMEM = -3,    /* workspace allocation failed */
+    VRAR_ECUDA = -4,     /* a CUDA runtime call failed (no device, launch error, ...) */
+    VRAR_ETIMEDOUT = -5  /* a device wait hit its time limit (reported by vrar_query_status) */
+};
+
+/*
+ * All-reduce. On return of the stream, every rank_out[p] (n elements) holds
+ * the element-wise sum over ranks of rank_in[0..P-1] (n elements each); all P
+ * outputs are bitwise identical. The order of the binary32 adds is fixed per
+ * algorithm:
+ *   ONESHOT, TWOSTAGE, TWOSTAGE_WRITE: ascending rank order from rank 0, one
+ *     rounding to the element type at the end ([CAR] Summary; the order is
+ *     this library's choice, the page fixes none).
+ *   RD (P = 2^m): m steps; at step k rank p adds its partner p XOR 2^k's
+ *     current partial to its own and rounds to the element type
+ *     ([NVRAR] phase 2, "Fused Payloads").
+ *   HIER (P = G*L, rank r = g*L + l): ascending sum over the L ranks of group
+ *     g, one rounding; then RD across the G groups; then copy to the group
+ *     ([NVRAR] phases 1-3). L is set by vrar_set_group_size.
+ *   AUTO: the algorithm vrar_select_algo returns, unless the environment
+ *     variable VRAR_ALGO (oneshot|twostage|twostage_write|rd|hier) names one.
+ */
+VRAR_API int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, size_t n,
+                            vrar_dtype_t dtype, vrar_algo_t algo, vrar_stream_t stream);
+
+/*
+ * Reduce-scatter ([NVRAR] phase 1 over one group of P ranks). rank_in[p] has
+ * n elements; rank_out[p] has n / P elements and receives elements
+ * [p*n/P, (p+1)*n/P) of the ascending-rank sum. Requires n % P == 0.
+ */
+VRAR_API int vrar_reduce_scatter(const void* const rank_in[], void* const rank_out[], int P, size_t n,
+                                 vrar_dtype_t dtype, vrar_stream_t stream);
+
+/*
+ * All-gather ([NVRAR] phase 3 over one group of P ranks). rank_in[p] has
+ * n / P elements; rank_out[p] has n elements and receives
+ * rank_in[0] | rank_in[1] | ... | rank_in[P-1] (exact copies). Requires
+ * n % P == 0.
+ */
+VRAR_API int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, size_t n,
+                             vrar_dtype_t dtype, vrar_stream_t stream);
+
+/*
+ * The algorithm VRAR_ALGO_AUTO uses for (P, n, dtype) on the current device:
+ * a table of per-size crossovers measured on a B200, in the spirit of the
+ * size gates the sources show ([CAR] "Scope of impact": write mode only above
+ * 4 MiB at 8 ranks). Never returns an algorithm that rejects the shape.
+ * Returns a vrar_algo_t value, or VRAR_EINVAL.
+ */
+VRAR_API int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype);
+
+/* Group size L used by VRAR_ALGO_HIER (default 8). Returns VRAR_OK or
+ * VRAR_EINVAL (L < 1 or L > VRAR_MAX_RANKS). Process-wide setting. */
+VRAR_API int vrar_set_group_size(int L);
+VRAR_API int vrar_get_group_size(void);
+
+/* Chunk count C of the recursive-doubling exchange (default 4): every thread
+ * keeps C payload pieces in flight per step ([NVRAR] "Chunked Non-blocking
+ * Communication"). Results do not depend on C. Range 1..8. */
+VRAR_API int vrar_set_rd_chunks(int C);
+VRAR_API int vrar_get_rd_chunks(void);
+
+/* Whether ONESHOT / TWOSTAGE / TWOSTAGE_WRITE run the start and end flag
+ * barriers of [CAR] (default 1 = yes). Inside one launch on one device the
+ * kernel boundary already orders the calls, so 0 drops them; the 2-stage mid
+ * barrier always runs because the all-gather reads other ranks' results. */
+VRAR_API int vrar_set_edge_sync(int on);
+VRAR_API int vrar_get_edge_sync(void);
+
+/* Time limit of every device wait, in nanoseconds of %globaltimer
+ * (default 2e9). Range 1e5 .. 6e10. */
+VRAR_API int vrar_set_spin_timeout_ns(uint64_t ns);
+VRAR_API uint64_t vrar_get_spin_timeout_ns(void);
+
+/*
+ * Wait for `stream`, then return and clear the device status word of the
+ * current device: VRAR_OK, or VRAR_ETIMEDOUT if any wait of any call since
+ * the last query ran out of time. If info is not NULL it receives details of
+ * the first failure: info[0] = call sequence number, info[1] = phase
+ * (1 start, 2 mid, 3 end, 4 payload), info[2] = waiting rank, info[3] = block.
+ */
+VRAR_API int vrar_query_status(vrar_stream_t stream, uint32_t info[4]);
+
+/* Grow the current device's workspace now to at least `bytes` of payload
+ * slots (so that later calls, e.g. under stream capture, need not allocate).
+ * vrar_workspace_bytes returns the payload-slot bytes a call would need. */
+VRAR_API int vrar_reserve(size_t bytes);
+VRAR_API size_t vrar_workspace_bytes(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t algo);
+
+/* Free the current device's workspace (synchronises the device). The next
+ * call allocates a fresh, zeroed one. */
+VRAR_API int vrar_reset(void);
+
+/* Testing aid: ranks whose bit is set skip every flag post and payload send
+ * of the following calls (until set back to 0), so that their peers' waits
+ * run out of time and report VRAR_ETIMEDOUT instead of hanging. */
+VRAR_API int vrar_debug_set_fault_mask(uint32_t mask);
+
+/* Static description of a return code. */
+VRAR_API const char* vrar_strerror(int code);
+
+VRAR_API int vrar_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VRAR_H */

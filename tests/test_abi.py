@@ -1,0 +1,138 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol include/vrar.h
+declares, and rejects bad arguments on the host before touching a device.
+
+No compute call reaches a kernel here. The pointers below are fake device
+addresses; every call that uses them fails its host-side checks first, except
+the one test that needs "no device" and is skipped when a GPU is present.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import collective_all_reduce_virtual_b200 as vrar
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "vrar.h")
+L = vrar.lib()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    return set(re.findall(r"^VRAR_API\s+[\w\s\*]+?\b(vrar_\w+)\(", src, flags=re.M))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    declared = header_functions()
+    assert len(declared) >= 19
+    assert declared == set(vrar.SIGNATURES), "binding signatures and header declarations differ"
+    for name in declared:
+        assert hasattr(L, name), f"{name} not exported by libvrar.so"
+
+
+def test_version_and_strerror():
+    assert vrar.version() == 1
+    for code, word in ((0, "success"), (-1, "invalid"), (-2, "not supported"), (-3, "allocation"),
+                       (-4, "CUDA"), (-5, "timed out"), (-99, "unknown")):
+        assert word in vrar.strerror(code)
+
+
+def _ptrs(base, P, stride=1 << 20):
+    return vrar.ptr_array([base + p * stride for p in range(P)])
+
+
+IN, OUT = 0x7F0000000000, 0x7F1000000000
+
+
+def call_ar(ins, outs, P, n, dtype=0, algo=1):
+    return L.vrar_allreduce(ins, outs, P, n, dtype, algo, None)
+
+
+def test_rejects_bad_rank_counts_and_dtypes():
+    assert call_ar(_ptrs(IN, 1), _ptrs(OUT, 1), 0, 16) == vrar.EINVAL
+    assert call_ar(_ptrs(IN, 33), _ptrs(OUT, 33), 33, 16) == vrar.EINVAL
+    assert call_ar(_ptrs(IN, 2), _ptrs(OUT, 2), 2, 16, dtype=7) == vrar.EINVAL
+    assert call_ar(_ptrs(IN, 2), _ptrs(OUT, 2), 2, 16, algo=9) == vrar.EINVAL
+    assert L.vrar_allreduce(None, _ptrs(OUT, 2), 2, 16, 0, 1, None) == vrar.EINVAL
+
+
+def test_rejects_null_and_misaligned_pointers():
+    ins = vrar.ptr_array([IN, 0])
+    assert call_ar(ins, _ptrs(OUT, 2), 2, 16) == vrar.EINVAL
+    ins = vrar.ptr_array([IN, IN + (1 << 20) + 8])  # 8-byte aligned only
+    assert call_ar(ins, _ptrs(OUT, 2), 2, 16) == vrar.EINVAL
+
+
+def test_rejects_overlap():
+    # out[1] overlaps in[0]
+    outs = vrar.ptr_array([OUT, IN + 16])
+    assert call_ar(_ptrs(IN, 2), outs, 2, 64) == vrar.EINVAL
+    # two outputs overlap each other
+    outs = vrar.ptr_array([OUT, OUT + 32])
+    assert call_ar(_ptrs(IN, 2), outs, 2, 64) == vrar.EINVAL
+
+
+def test_shape_errors():
+    assert call_ar(_ptrs(IN, 3), _ptrs(OUT, 3), 3, 16, algo=4) == vrar.ENOTSUP  # RD needs 2^k
+    vrar.set_group_size(4)
+    try:
+        assert call_ar(_ptrs(IN, 12), _ptrs(OUT, 12), 12, 16, algo=5) == vrar.ENOTSUP  # G = 3
+        assert call_ar(_ptrs(IN, 6), _ptrs(OUT, 6), 6, 16, algo=5) == vrar.ENOTSUP  # 4 does not divide 6
+    finally:
+        vrar.set_group_size(8)
+    # reduce-scatter / all-gather need n % P == 0
+    assert L.vrar_reduce_scatter(_ptrs(IN, 3), _ptrs(OUT, 3), 3, 10, 0, None) == vrar.EINVAL
+    assert L.vrar_all_gather(_ptrs(IN, 3), _ptrs(OUT, 3), 3, 10, 0, None) == vrar.EINVAL
+
+
+def test_zero_length_is_a_no_op():
+    assert call_ar(_ptrs(IN, 4), _ptrs(OUT, 4), 4, 0) == vrar.OK
+
+
+# These calls pass every host check, so on a machine with a GPU they would
+# launch a kernel on fake addresses: they run only where there is no device.
+@pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a GPU")
+def test_valid_call_without_device_reports_cuda_error():
+    assert call_ar(_ptrs(IN, 2), _ptrs(OUT, 2), 2, 64) == vrar.ECUDA
+    # adjacent, non-overlapping ranges pass the overlap check
+    assert call_ar(vrar.ptr_array([IN, IN + 128]), _ptrs(OUT, 2), 2, 64) == vrar.ECUDA
+
+
+def test_settings_round_trip_and_ranges():
+    assert vrar.get_group_size() == 8 and vrar.get_rd_chunks() == 4 and vrar.get_edge_sync()
+    for bad in (0, 33):
+        with pytest.raises(vrar.VrarError):
+            vrar.set_group_size(bad)
+    for bad in (0, 9):
+        with pytest.raises(vrar.VrarError):
+            vrar.set_rd_chunks(bad)
+    with pytest.raises(vrar.VrarError):
+        vrar.set_spin_timeout_ns(10)
+    t = vrar.get_spin_timeout_ns()
+    vrar.set_spin_timeout_ns(5_000_000)
+    assert vrar.get_spin_timeout_ns() == 5_000_000
+    vrar.set_spin_timeout_ns(t)
+    vrar.set_edge_sync(False)
+    assert not vrar.get_edge_sync()
+    vrar.set_edge_sync(True)
+
+
+def test_selector_is_defined_for_every_shape():
+    for P in range(1, 33):
+        for n in (1, 1000, 65536, 1 << 20, 117440512):
+            for dt in (torch.bfloat16, torch.float32):
+                a = vrar.select_algo(P, n, dt)
+                assert a in ("oneshot", "twostage", "twostage_write", "rd", "hier")
+                if a == "rd":
+                    assert P & (P - 1) == 0
+
+
+def test_workspace_bytes():
+    # RD at P=8 on 2 MiB of bf16 per rank: 8 ranks x 3 steps x 131072 items x 32 bytes
+    assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 8 * 3 * 131072 * 32
+    # HIER 4 x 8 on 2 MiB: 32 ranks x 2 steps x (131072 / 8) items x 32 bytes
+    assert vrar.workspace_bytes(32, 1 << 20, torch.bfloat16, "hier") == 32 * 2 * 16384 * 32
+    assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "oneshot") == 0
+    assert vrar.workspace_bytes(3, 1 << 20, torch.bfloat16, "rd") == 0

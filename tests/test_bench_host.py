@@ -1,0 +1,94 @@
+"""Host logic of bench.py on the CPU: bandwidth arithmetic, buffer rotation,
+clock parsing, and the multi-rank timing reduction on 2 gloo ranks."""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_busbw_and_bytes():
+    # 1 MiB per rank at P=8 in 10 us: algbw 104.8576 GB/s, busbw x 2*7/8
+    assert bench.busbw_gbs(8, 524288, 2, 10e-6) == pytest.approx(1048576 / 10e-6 * 1.75 / 1e9)
+    assert bench.busbw_gbs(1, 100, 4, 1.0) == pytest.approx(400 / 1e9)
+    assert bench.b_min_bytes(8, 524288, 2) == 16 * 1024 * 1024
+
+
+def test_rotation_exceeds_l2():
+    for set_bytes in (2 << 20, 16 << 20, 128 << 20, 3758096384):
+        R = bench.rotation_sets(set_bytes)
+        assert R >= 1
+        assert R * set_bytes >= min(3 * bench.L2_BYTES, set_bytes * 64) or set_bytes > 3 * bench.L2_BYTES
+
+
+def test_parse_clocks():
+    text = "\n".join([
+        "0, 1965 MHz, 1965 MHz, 650.10 W, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800 MHz, 1965 MHz, 990.00 W, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 345 MHz, 1965 MHz, 120.00 W, 0x0000000000000001, Not Active, Not Active, Not Active, Not Active",
+    ])
+    c = bench.parse_clocks_csv(text)
+    assert c["sm_mhz"] == pytest.approx(1882.5)
+    assert c["sm_max_mhz"] == 1965
+    assert c["reasons"] == ["sw_power_cap"]
+    assert c["samples"] == 3 and c["samples_under_load"] == 2
+
+
+def test_peaks_fallback(tmp_path):
+    assert bench.load_peaks(str(tmp_path / "missing.json")) == (bench.FALLBACK_HBM_GBS, "fallback")
+    p = tmp_path / "p.json"
+    p.write_text('{"hbm_gbs": 6451.5}')
+    assert bench.load_peaks(str(p)) == (6451.5, "measured")
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        m = bench.max_over_ranks(1.5 + rank, world)
+        q.put((rank, m))
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == {0: 2.5, 1: 2.5}
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.run_reference(bench.argparse.Namespace(steps=3, warmup=3)) is None
+
+
+def test_reference_arm_line_on_cpu(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3"])
+    line = bench.json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["metric"] == bench.METRIC

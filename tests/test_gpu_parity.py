@@ -1,0 +1,332 @@
+"""GPU path against the CPU oracle, through the C ABI (Python binding).
+
+Bit-exact: every algorithm fixes its fp32-accumulate order, and the oracle
+restates that order, so outputs must match bit for bit (NaN never appears in
+these inputs). The fp64 tolerances (bf16 1e-2, fp32 1e-5, relative to the sum
+of magnitudes) are checked as well.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from util import TORCH_DT, bits_of, from_np, gen, hexvals, load_golden, parse_algo, to_np
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import collective_all_reduce_virtual_b200 as vrar
+else:  # collected on the CPU machine, never run there
+    vrar = None
+
+RTOL = {"bf16": 1e-2, "fp32": 1e-5}
+
+
+@pytest.fixture(autouse=True)
+def _defaults():
+    yield
+    if vrar is not None:
+        vrar.set_group_size(8)
+        vrar.set_rd_chunks(4)
+        vrar.set_edge_sync(True)
+        vrar.set_spin_timeout_ns(2_000_000_000)
+        vrar.debug_set_fault_mask(0)
+
+
+def _dev(xs_np, dtype):
+    return [from_np(x, dtype).cuda() for x in xs_np]
+
+
+def run(algo, xs_np, dtype, L=8, C=4, edge=True):
+    vrar.set_group_size(L)
+    vrar.set_rd_chunks(C)
+    vrar.set_edge_sync(edge)
+    outs = vrar.all_reduce(_dev(xs_np, dtype), algo=algo)
+    rc, info = vrar.query_status()
+    assert rc == 0, f"device status {rc} {info}"
+    return [to_np(o) for o in outs]
+
+
+def assert_bits(got, want, what):
+    for p, (g, w) in enumerate(zip(got, want)):
+        if not np.array_equal(bits_of(g), bits_of(w)):
+            bad = np.nonzero(bits_of(g) != bits_of(w))[0]
+            raise AssertionError(f"{what}: rank {p} differs at {bad[:8]} (of {bad.size})")
+
+
+def algos_for(P):
+    out = [("oneshot", 8), ("twostage", 8), ("twostage_write", 8)]
+    if P & (P - 1) == 0:
+        out.append(("rd", 8))
+        for L in sorted({1, max(1, P // 2), P}):
+            out.append(("hier", L))
+    return out
+
+
+# ---- small shapes: several CTAs' worth of items and a ragged tail ----------------------------
+
+SHAPES = [(P, n) for P in (1, 2, 3, 4, 5, 8) for n in (1, 7, 8, 9, 4099, 100_003)] + \
+         [(P, n) for P in (16, 32) for n in (1, 9, 20_011)]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("P,n", SHAPES)
+def test_parity_small(P, n, dtype):
+    xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P * 1000 + n)
+    for algo, L in algos_for(P):
+        want = oracle.allreduce(algo, xs, dtype, L=L, chunks=4)
+        got = run(algo, xs, dtype, L=L)
+        assert_bits(got, want, f"{algo} L={L} P={P} n={n} {dtype}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_integer_inputs_give_exact_sums(dtype):
+    for P in (2, 4, 8, 16, 32):
+        n = 5003
+        xs = gen(P, n, dtype, synth.INT8, seed=P)
+        exact = np.stack([oracle.to_float(x, dtype) for x in xs]).astype(np.int64).sum(axis=0)
+        for algo, L in algos_for(P):
+            got = run(algo, xs, dtype, L=L)
+            for g in got:
+                assert (oracle.to_float(g, dtype) == exact).all(), f"{algo} L={L} P={P}"
+
+
+def test_golden_order_cases_on_gpu():
+    for case in load_golden()["cases"]:
+        dt = case["dtype"]
+        xs = [hexvals(row, dt) for row in case["inputs"]]
+        for spec, want_strs in case["expect"].items():
+            algo, L = parse_algo(spec)
+            want = hexvals(want_strs, dt)
+            got = run(algo, xs, dt, L=L if L is not None else 8)
+            assert_bits(got, [want] * len(got), f"{case['name']} {spec}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_fp64_tolerance(dtype):
+    for P in (2, 8, 32):
+        xs = gen(P, 30_000, dtype, synth.normal(0.0, 1.0), seed=77 + P)
+        S, A = oracle.fp64_reference(xs, dtype)
+        for algo, L in algos_for(P):
+            y = oracle.to_float(run(algo, xs, dtype, L=L)[0], dtype)
+            assert (np.abs(y - S) <= RTOL[dtype] * A).all(), f"{algo} L={L} P={P}"
+
+
+def test_special_values_classes():
+    """inf, -inf, subnormals and signed zeros (NaN only as inf - inf)."""
+    vals = np.array([np.inf, -np.inf, 1e-40, -1e-40, 0.0, -0.0, 3e38, 3e38], np.float32)
+    xs32 = [vals, np.array([1.0, 1.0, 1e-40, 0.0, -0.0, -0.0, 3e38, -3e38], np.float32),
+            np.array([-np.inf, 2.0, 0.0, -1e-40, -0.0, -0.0, 0.0, 1.0], np.float32)]
+    for dtype in ("fp32", "bf16"):
+        xs = xs32 if dtype == "fp32" else [oracle.bf16_round(x) for x in xs32]
+        for algo in ("oneshot", "twostage", "twostage_write"):
+            want = oracle.allreduce(algo, xs, dtype)
+            got = run(algo, xs, dtype)
+            for g, w in zip(got, want):
+                gf, wf = oracle.to_float(g, dtype), oracle.to_float(w, dtype)
+                assert np.array_equal(np.isnan(gf), np.isnan(wf))
+                fin = ~np.isnan(wf)
+                assert np.array_equal(bits_of(g)[fin], bits_of(w)[fin]), f"{algo} {dtype}"
+
+
+# ---- the workload shapes at full size ---------------------------------------------------------
+
+def test_config_p2_ints_oneshot_and_rd():
+    xs = gen(2, 65_536, "bf16", synth.INT8, seed=0)
+    exact = np.stack([oracle.to_float(x, "bf16") for x in xs]).astype(np.int64).sum(axis=0)
+    for algo in ("oneshot", "rd"):
+        got = run(algo, xs, "bf16")
+        assert_bits(got, oracle.allreduce(algo, xs, "bf16"), algo)
+        assert (oracle.to_float(got[0], "bf16") == exact).all()
+        assert_bits(got, [got[0]] * 2, f"{algo} ranks equal")
+
+
+def test_config_p8_decode_1mib():
+    xs = gen(8, 64 * 8192, "bf16", synth.normal(0.0, 1.0), seed=0)
+    one = None
+    for algo in ("oneshot", "twostage", "twostage_write", "rd", "auto"):
+        want = oracle.allreduce(algo if algo != "auto" else vrar.select_algo(8, 64 * 8192), xs, "bf16")
+        got = run(algo, xs, "bf16")
+        assert_bits(got, want, algo)
+        if algo == "oneshot":
+            one = got
+        elif algo in ("twostage", "twostage_write"):
+            assert_bits(got, one, f"{algo} == oneshot")
+
+
+@pytest.mark.parametrize("n", [65_536, 131_072, 262_144, 524_288, 1_048_576])
+def test_config_p8_rd_sweep(n):
+    xs = gen(8, n, "bf16", synth.normal(0.0, 1.0), seed=0)
+    got = run("rd", xs, "bf16", C=4)
+    assert_bits(got, oracle.allreduce("rd", xs, "bf16", chunks=4), f"rd n={n}")
+
+
+def test_config_p8_rd_1000_calls_reuse_flags():
+    n = 262_144
+    xs = gen(8, n, "bf16", synth.normal(0.0, 1.0), seed=3)
+    want = oracle.allreduce("rd", xs, "bf16", chunks=4)
+    d_in = _dev(xs, "bf16")
+    outs = [torch.empty_like(t) for t in d_in]
+    vrar.set_rd_chunks(4)
+    for i in range(1000):
+        vrar.all_reduce(d_in, outs, algo="rd")
+        if i in (0, 499, 999):
+            assert_bits([to_np(o) for o in outs], want, f"call {i}")
+    rc, info = vrar.query_status()
+    assert rc == 0, info
+
+
+def test_cuda_graph_replay_reuses_flags():
+    n = 131_072
+    xs = gen(8, n, "bf16", synth.normal(0.0, 1.0), seed=4)
+    d_in = _dev(xs, "bf16")
+    for algo in ("rd", "twostage", "oneshot", "twostage_write"):
+        outs = [torch.empty_like(t) for t in d_in]
+        want = oracle.allreduce(algo, xs, "bf16")
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            vrar.all_reduce(d_in, outs, algo=algo, stream=s)  # sizes the workspace before capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(10):
+                vrar.all_reduce(d_in, outs, algo=algo)
+        for _ in range(50):
+            g.replay()
+        torch.cuda.synchronize()
+        rc, info = vrar.query_status()
+        assert rc == 0, (algo, info)
+        assert_bits([to_np(o) for o in outs], want, f"{algo} after 500 graph-replayed calls")
+        del g
+
+
+@pytest.mark.parametrize("n", [131_072, 1_048_576])
+def test_config_p32_hier_4x8(n):
+    xs = gen(32, n, "bf16", synth.uniform(-1.0, 1.0), seed=0)
+    got = run("hier", xs, "bf16", L=8)
+    assert_bits(got, oracle.allreduce("hier", xs, "bf16", L=8), f"hier 4x8 n={n}")
+
+
+@pytest.mark.slow
+def test_config_p8_prefill_sampled():
+    """16384 x 7168 bf16 per rank (1.88 GB of inputs): the 2-stage kernels on the
+    full size, checked on sampled outputs (every output element depends only on
+    the P inputs at the same index) and for equality of all P outputs."""
+    P, n = 8, 16384 * 7168
+    d_in = synth.make_inputs(P, n, torch.bfloat16, synth.normal(0.0, 0.02), seed=0, device="cuda",
+                             block=1 << 25)
+    rng = np.random.default_rng(0)
+    piece = (n // 8 + P - 1) // P * 8
+    edges = np.concatenate([np.arange(0, 64), n - 64 + np.arange(64)] +
+                           [np.arange(s * piece - 8, s * piece + 8) for s in range(1, P)])
+    idx = np.unique(np.concatenate([rng.integers(0, n, 200_000), edges]))
+    idx_t = torch.from_numpy(idx).cuda()
+    xs_s = [to_np(t[idx_t]) for t in d_in]
+    for algo in ("twostage", "twostage_write"):
+        outs = vrar.all_reduce(d_in, algo=algo)
+        rc, info = vrar.query_status()
+        assert rc == 0, info
+        want = oracle.allreduce(algo, xs_s, "bf16")
+        assert_bits([to_np(o[idx_t]) for o in outs], want, f"{algo} sampled")
+        for p in range(1, P):
+            assert torch.equal(outs[p].view(torch.int16), outs[0].view(torch.int16)), f"{algo} rank {p}"
+        del outs
+    torch.cuda.empty_cache()
+
+
+# ---- protocol properties ----------------------------------------------------------------------
+
+def test_chunk_count_and_edge_sync_do_not_change_results():
+    xs = gen(8, 50_001, "bf16", synth.normal(0.0, 1.0), seed=11)
+    ref = run("rd", xs, "bf16", C=1)
+    for C in range(2, 9):
+        assert_bits(run("rd", xs, "bf16", C=C), ref, f"rd C={C}")
+    ref = run("hier", xs, "bf16", L=2, C=1)
+    for C in (2, 4, 8):
+        assert_bits(run("hier", xs, "bf16", L=2, C=C), ref, f"hier C={C}")
+    for algo in ("oneshot", "twostage", "twostage_write"):
+        assert_bits(run(algo, xs, "bf16", edge=False), run(algo, xs, "bf16", edge=True), algo)
+
+
+def test_shapes_interleaved_across_calls():
+    """Flags and payload slots are reused across calls of different P, n and
+    algorithm without ever being cleared."""
+    plan = [(8, 70_000, "twostage", 8), (32, 40_000, "hier", 8), (2, 9, "rd", 8), (8, 70_000, "rd", 8),
+            (4, 100_000, "oneshot", 8), (32, 40_000, "hier", 4), (16, 33_333, "twostage_write", 8),
+            (8, 70_000, "twostage", 8)]
+    for i, (P, n, algo, L) in enumerate(plan * 2):
+        xs = gen(P, n, "bf16", synth.normal(0.0, 1.0), seed=i)
+        assert_bits(run(algo, xs, "bf16", L=L), oracle.allreduce(algo, xs, "bf16", L=L), f"step {i} {algo}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_reduce_scatter_and_all_gather(dtype):
+    for P in (1, 2, 3, 8, 32):
+        for m in (8, 37, 4104, 20_000):
+            n = m * P
+            xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P + m)
+            got = [to_np(o) for o in vrar.reduce_scatter(_dev(xs, dtype))]
+            assert_bits(got, oracle.reduce_scatter(xs, dtype), f"RS P={P} m={m}")
+            sl = gen(P, m, dtype, synth.normal(0.0, 1.0), seed=P * m)
+            got = [to_np(o) for o in vrar.all_gather(_dev(sl, dtype))]
+            assert_bits(got, oracle.all_gather(sl, dtype), f"AG P={P} m={m}")
+    rc, info = vrar.query_status()
+    assert rc == 0, info
+
+
+def test_workspace_growth_between_calls():
+    vrar.reset()
+    for n in (1000, 300_000, 1_000, 2_000_000):
+        xs = gen(8, n, "bf16", synth.normal(0.0, 1.0), seed=n)
+        assert_bits(run("rd", xs, "bf16"), oracle.allreduce("rd", xs, "bf16"), f"rd n={n}")
+
+
+def test_device_argument_errors():
+    t = torch.zeros(1024, dtype=torch.bfloat16, device="cuda")
+    ins = [t[:256], t[256:512]]
+    outs = [t[512:768], t[520:776]]  # overlapping outputs
+    with pytest.raises(vrar.VrarError) as e:
+        vrar.all_reduce(ins, outs, algo="oneshot")
+    assert e.value.code == vrar.EINVAL
+    mis = [t[1:257], t[257:513]]  # 2-byte offset: not 16-byte aligned
+    with pytest.raises(vrar.VrarError) as e:
+        vrar.all_reduce(mis, algo="oneshot")
+    assert e.value.code == vrar.EINVAL
+    with pytest.raises(vrar.VrarError) as e:
+        vrar.all_reduce([t[:256]] * 3, algo="rd")
+    assert e.value.code in (vrar.EINVAL, vrar.ENOTSUP)
+
+
+# ---- failure detection: bounded waits, no GPU fault ----------------------------------------------
+
+@pytest.mark.parametrize("algo,P,L,edge,phase", [
+    ("oneshot", 4, 8, True, 1),
+    ("twostage", 4, 8, False, 2),
+    ("twostage_write", 8, 8, True, 1),
+    ("rd", 4, 8, True, 4),
+    ("hier", 8, 2, True, 4),
+])
+def test_missing_rank_times_out_and_recovers(algo, P, L, edge, phase):
+    """A rank that never posts (fault mask) makes its peers' waits run out; the
+    kernel records VRAR_ETIMEDOUT and exits, and the next call works."""
+    xs = gen(P, 40_000, "bf16", synth.normal(0.0, 1.0), seed=5)
+    d_in = _dev(xs, "bf16")
+    vrar.set_group_size(L)
+    vrar.set_edge_sync(edge)
+    vrar.set_spin_timeout_ns(50_000_000)
+    vrar.debug_set_fault_mask(1 << 1)
+    vrar.all_reduce(d_in, algo=algo)
+    rc, info = vrar.query_status()
+    assert rc == vrar.ETIMEDOUT, (rc, info)
+    assert info[1] == phase
+    vrar.debug_set_fault_mask(0)
+    outs = vrar.all_reduce(d_in, algo=algo)
+    rc, info = vrar.query_status()
+    assert rc == 0, info
+    assert_bits([to_np(o) for o in outs], oracle.allreduce(algo, xs, "bf16", L=L), f"{algo} after timeout")
