@@ -26,16 +26,18 @@
 namespace vrar {
 
 constexpr int kMaxRanks = 32;
-constexpr int kThreads = 512;          // threads per CTA of every kernel
+#ifndef VRAR_THREADS
+#define VRAR_THREADS 512
+#endif
+constexpr int kThreads = VRAR_THREADS;  // threads per CTA of every kernel
 constexpr int kMaxCtas = 2048;         // grid cap; sizes the signal arrays
 constexpr int kSigPhaseWords = kMaxCtas * kMaxRanks;
 constexpr int kPhases = 3;             // start, mid, end
 
-// Control words at the start of the workspace.
+// Control words at the start of the workspace (32-bit words).
 enum Ctrl : int {
-  kStatus = 0,     // sticky error code (0 = none) until the host reads it
-  kEpoch = 1,      // sequence number of the last completed call
-  kDone = 2,       // CTAs of the running call that have finished
+  kTicket = 0,     // 64-bit ticket (words 0-1): high half = calls completed, low half = CTAs arrived
+  kStatus = 2,     // sticky error code (0 = none) until the host reads it
   kFailEpoch = 3,  // sequence number of a call in which some wait gave up
   kInfo = 4,       // 4 words: failing call, phase, rank, block
   kCtrlWords = 16
@@ -275,7 +277,27 @@ __device__ __forceinline__ uint4 reduce_item(const RankPtrs& rp, int first, int 
   return acc.round();
 }
 
-// ---- per-CTA protocol state ----------------------------------------------------------
+// ---- launch ordering -------------------------------------------------------------------
+// Kernels are launched with programmatic stream serialisation: the next call's
+// grid may be scheduled while this one drains, and it waits in
+// griddepcontrol.wait until this grid has completed and its memory is visible.
+// Every kernel executes pdl_wait() before its first global memory access.
+// A grid's dependents launch only once all its CTAs have triggered, i.e. once
+// they are all resident, so the co-residency the waits below rely on holds.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---- per-call sequence number [NVRAR "Sequence-Number Synchronization"] ------------------
+// One 64-bit ticket per device: every CTA of a call adds 1 (a relaxed atomic:
+// the ticket is the only location involved, and its modification order
+// serialises the adds). The CTA that sees the low half reach gridDim.x - 1 is
+// the last to arrive, and adds 2^32 - gridDim.x: the call count goes up by one
+// and the arrival count back to 0, for the next launch (stream order). Every
+// CTA of a call therefore reads the same call count c and uses c + 1 as the
+// call's flag; flags grow by one per call that uses them, so a flag or payload
+// word left by any earlier call never equals the current flag (until 2^32
+// calls wrap it). Kernels that use no flags never touch the ticket.
 
 struct Cta {
   int r;          // virtual rank this CTA acts for
@@ -283,33 +305,35 @@ struct Cta {
   uint32_t flag;  // this call's sequence number (never 0)
 };
 
-__device__ __forceinline__ Cta cta_begin(const KArgs& a) {
-  __shared__ uint32_t s_flag;
-  if (threadIdx.x == 0) {
-    uint32_t f = ld_relaxed(a.ctrl + kEpoch) + 1u;
-    s_flag = f == 0u ? 1u : f;  // 0 is the value of a never-written word
-  }
-  __syncthreads();
+__device__ __forceinline__ Cta cta_coords(const KArgs& a) {
   Cta c;
   c.r = static_cast<int>(blockIdx.x % a.P);
   c.b = static_cast<int>(blockIdx.x / a.P);
-  c.flag = s_flag;
+  c.flag = 0;
   return c;
 }
 
-// Every CTA counts itself out; the last one publishes this call's sequence
-// number for the next call (stream order makes it visible there) and resets
-// the counter. acq_rel orders each CTA's earlier read of kEpoch before its
-// count, so no CTA of this call can see the new value.
-__device__ __forceinline__ void cta_end(const KArgs& a, const Cta& c) {
-  __syncthreads();
+// Thread 0 takes the ticket (issue this early: the result is needed only by
+// cta_publish_flag, so the atomic's latency overlaps the first data loads).
+__device__ __forceinline__ unsigned long long cta_take_ticket(const KArgs& a) {
+  unsigned long long old = 0;
   if (threadIdx.x == 0) {
-    const uint32_t old = atom_add_acq_rel(a.ctrl + kDone, 1u);
-    if (old == gridDim.x - 1) {
-      st_relaxed(a.ctrl + kDone, 0u);
-      st_relaxed(a.ctrl + kEpoch, c.flag);
-    }
+    unsigned long long* t = reinterpret_cast<unsigned long long*>(a.ctrl + kTicket);
+    old = atomicAdd(t, 1ull);
+    if (static_cast<uint32_t>(old) == gridDim.x - 1) atomicAdd(t, (1ull << 32) - gridDim.x);
   }
+  return old;
+}
+
+// Broadcast the call's flag to the whole CTA (contains a CTA barrier).
+__device__ __forceinline__ void cta_publish_flag(Cta& c, unsigned long long ticket) {
+  __shared__ uint32_t s_flag;
+  if (threadIdx.x == 0) {
+    const uint32_t f = static_cast<uint32_t>(ticket >> 32) + 1u;
+    s_flag = f == 0u ? 1u : f;  // 0 is the value of a never-written word
+  }
+  __syncthreads();
+  c.flag = s_flag;
 }
 
 __device__ __noinline__ void report_timeout(const KArgs& a, const Cta& c, uint32_t phase) {

@@ -29,16 +29,18 @@ __device__ __forceinline__ int64_t lo_of(int64_t part, int64_t piece, int64_t to
 // time, so all but the first read of each line hit L2.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_oneshot(const KArgs a) {
-  const Cta c = cta_begin(a);
-  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
-  bool ok = !a.edge_sync || block_barrier(a, c, kPhStart);
-  if (ok) {
-    void* out = a.ptr.out[c.r];
-    for (int64_t it = static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < a.items; it += stride)
-      store_item<D, true>(out, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
-    if (a.edge_sync) block_barrier(a, c, kPhEnd);
+  pdl_wait();
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  if (a.edge_sync) {
+    cta_publish_flag(c, cta_take_ticket(a));
+    if (!block_barrier(a, c, kPhStart)) return;
   }
-  cta_end(a, c);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  void* out = a.ptr.out[c.r];
+  for (int64_t it = static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < a.items; it += stride)
+    store_item<D, true>(out, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
+  if (a.edge_sync) block_barrier(a, c, kPhEnd);
 }
 
 // 2-stage [CAR "cross_device_reduce_2stage"], pull mode. Stage 1: rank r
@@ -46,41 +48,44 @@ __global__ void __launch_bounds__(kThreads) k_oneshot(const KArgs a) {
 // barrier. Stage 2: rank r copies every other slice s out of out[s].
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_twostage(const KArgs a) {
-  const Cta c = cta_begin(a);
+  pdl_wait();
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const unsigned long long ticket = cta_take_ticket(a);
+  if (a.edge_sync) {
+    cta_publish_flag(c, ticket);
+    if (!block_barrier(a, c, kPhStart)) return;
+  }
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
   const int64_t piece = (a.items + a.P - 1) / a.P;
-  bool ok = !a.edge_sync || block_barrier(a, c, kPhStart);
-  if (ok) {
+  void* own = a.ptr.out[c.r];
+  {
     const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
-    void* own = a.ptr.out[c.r];
     for (int64_t it = lo + t0; it < hi; it += stride)
       store_item<D, false>(own, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
-    ok = block_barrier(a, c, kPhMid);
   }
-  if (ok) {
-    void* own = a.ptr.out[c.r];
-    for (int64_t off = t0; off < piece; off += stride) {
-      // Up to 8 peer slices per batch so that the loads overlap; sources are
-      // staggered (r+1, r+2, ...) so the ranks do not all read one slice at once.
-      for (int j0 = 1; j0 < a.P; j0 += 8) {
-        uint4 v[8];
-        int64_t it[8];
+  if (!a.edge_sync) cta_publish_flag(c, ticket);
+  if (!block_barrier(a, c, kPhMid)) return;
+  for (int64_t off = t0; off < piece; off += stride) {
+    // Up to 8 peer slices per batch so that the loads overlap; sources are
+    // staggered (r+1, r+2, ...) so the ranks do not all read one slice at once.
+    for (int j0 = 1; j0 < a.P; j0 += 8) {
+      uint4 v[8];
+      int64_t it[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int s = (c.r + j0 + j) % a.P;
-          it[j] = s * piece + off;
-          if (j0 + j < a.P && it[j] < lo_of(s + 1, piece, a.items)) v[j] = load_item_peer<D>(a.ptr.out[s], it[j], a.n);
-          else it[j] = -1;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j0 + j < a.P && it[j] >= 0) store_item<D, true>(own, it[j], a.n, v[j]);
+      for (int j = 0; j < 8; ++j) {
+        const int s = (c.r + j0 + j) % a.P;
+        it[j] = s * piece + off;
+        if (j0 + j < a.P && it[j] < lo_of(s + 1, piece, a.items)) v[j] = load_item_peer<D>(a.ptr.out[s], it[j], a.n);
+        else it[j] = -1;
       }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j0 + j < a.P && it[j] >= 0) store_item<D, true>(own, it[j], a.n, v[j]);
     }
-    if (a.edge_sync) block_barrier(a, c, kPhEnd);
   }
-  cta_end(a, c);
+  if (a.edge_sync) block_barrier(a, c, kPhEnd);
 }
 
 // 2-stage write mode [CAR "cross_device_reduce_2stage_write_mode", Root cause
@@ -89,25 +94,27 @@ __global__ void __launch_bounds__(kThreads) k_twostage(const KArgs a) {
 // the end barrier's flags.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
-  const Cta c = cta_begin(a);
+  pdl_wait();
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  if (a.edge_sync) {
+    cta_publish_flag(c, cta_take_ticket(a));
+    if (!block_barrier(a, c, kPhStart)) return;
+  }
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t piece = (a.items + a.P - 1) / a.P;
-  bool ok = !a.edge_sync || block_barrier(a, c, kPhStart);
-  if (ok) {
-    const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
-    for (int64_t it = lo + static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < hi; it += stride) {
-      const uint4 v = reduce_item<D>(a.ptr, 0, a.P, it, a.n);
-      for (int j = 0; j < a.P; ++j) {
-        const int p = (c.r + j) % a.P;
-        store_item<D, true>(a.ptr.out[p], it, a.n, v);
-      }
-    }
-    if (a.edge_sync) {
-      __threadfence();
-      block_barrier(a, c, kPhEnd);
+  const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
+  for (int64_t it = lo + static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < hi; it += stride) {
+    const uint4 v = reduce_item<D>(a.ptr, 0, a.P, it, a.n);
+    for (int j = 0; j < a.P; ++j) {
+      const int p = (c.r + j) % a.P;
+      store_item<D, true>(a.ptr.out[p], it, a.n, v);
     }
   }
-  cta_end(a, c);
+  if (a.edge_sync) {
+    __threadfence();
+    block_barrier(a, c, kPhEnd);
+  }
 }
 
 // Recursive doubling with fused payload words [NVRAR phase 2, "Fused
@@ -158,12 +165,17 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
 
 template <class D, int C>
 __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
-  const Cta c = cta_begin(a);
+  pdl_wait();
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const unsigned long long ticket = cta_take_ticket(a);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
   const int64_t per_chunk = (a.items + C - 1) / C;
   bool ok = true;
-  for (int64_t base = 0; base < per_chunk && ok; base += stride) {
+  // The trip count is the same for every thread of the CTA (the flag is
+  // published inside the first trip, after that trip's input loads issue).
+  for (int64_t base = 0; base < per_chunk; base += stride) {
     const int64_t j = base + t0;
     uint4 v[C];
     int64_t idx[C];
@@ -171,9 +183,11 @@ __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       idx[k] = k * per_chunk + j;
-      val[k] = j < per_chunk && idx[k] < a.items;
+      val[k] = ok && j < per_chunk && idx[k] < a.items;
       if (val[k]) v[k] = load_item_input<D>(a.ptr.in[c.r], idx[k], a.n);
     }
+    if (base == 0) cta_publish_flag(c, ticket);
+    if (!ok) continue;
     ok = rd_exchange<D, C, false>(a, c, v, idx, val, a.items);
     if (ok) {
 #pragma unroll
@@ -181,7 +195,6 @@ __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
         if (val[k]) store_item<D, true>(a.ptr.out[c.r], idx[k], a.n, v[k]);
     }
   }
-  cta_end(a, c);
 }
 
 // Hierarchical all-reduce [NVRAR Methodology item 3, phases 1-3] with P = G*L
@@ -193,7 +206,10 @@ __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
 // L ranks of group g. Slices are cut into C chunks as in k_rd.
 template <class D, int C>
 __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
-  const Cta c = cta_begin(a);
+  pdl_wait();
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const unsigned long long ticket = cta_take_ticket(a);
   const int L = a.L, g = c.r / L, l = c.r % L;
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
@@ -201,7 +217,7 @@ __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
   const int64_t lo = lo_of(l, piece, a.items), len = lo_of(l + 1, piece, a.items) - lo;
   const int64_t per_chunk = (len + C - 1) / C;
   bool ok = true;
-  for (int64_t base = 0; base < per_chunk && ok; base += stride) {
+  for (int64_t base = 0; base < per_chunk; base += stride) {  // same trip count in the whole CTA
     const int64_t j = base + t0;
     uint4 v[C];
     int64_t idx[C];
@@ -209,9 +225,11 @@ __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       idx[k] = k * per_chunk + j;
-      val[k] = j < per_chunk && idx[k] < len;
+      val[k] = ok && j < per_chunk && idx[k] < len;
       if (val[k]) v[k] = reduce_item<D>(a.ptr, g * L, L, lo + idx[k], a.n);
     }
+    if (base == 0) cta_publish_flag(c, ticket);
+    if (!ok) continue;
     ok = rd_exchange<D, C, true>(a, c, v, idx, val, piece);
     if (ok) {
 #pragma unroll
@@ -224,7 +242,6 @@ __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
       }
     }
   }
-  cta_end(a, c);
 }
 
 // Standalone reduce-scatter [NVRAR phase 1 over one group]: rank p writes
@@ -233,6 +250,8 @@ __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
 // every slice starts on a 16-byte boundary), element path otherwise.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_reduce_scatter(const KArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int r = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(b) * kThreads + threadIdx.x;
@@ -256,6 +275,8 @@ __global__ void __launch_bounds__(kThreads) k_reduce_scatter(const KArgs a) {
 // reads its n/P elements once and streams them to offset s*m of all P outputs.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_all_gather(const KArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int s = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(b) * kThreads + threadIdx.x;

@@ -22,7 +22,7 @@ constexpr int kMaxDevices = 64;
 struct Settings {
   std::atomic<int> group_size{8};
   std::atomic<int> rd_chunks{4};
-  std::atomic<int> edge_sync{1};
+  std::atomic<int> edge_sync{0};
   std::atomic<uint64_t> timeout_ns{2000000000ull};
   std::atomic<uint32_t> fault_mask{0};
 };
@@ -225,10 +225,30 @@ KernelFn pick_kernel(vrar_algo_t algo, int C) {
 #undef VRAR_CHUNK_CASES
 }
 
+// Programmatic dependent launch is on unless VRAR_PDL=0 (read once).
+bool pdl_enabled() {
+  static int cached = -1;
+  if (cached < 0) {
+    const char* s = std::getenv("VRAR_PDL");
+    cached = (s && s[0] == '0') ? 0 : 1;
+  }
+  return cached == 1;
+}
+
 int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream) {
-  fn<<<grid, kThreads, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? VRAR_OK : VRAR_ECUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, a);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return VRAR_OK;
 }
 
 const char* algo_name(int a) {

@@ -155,9 +155,13 @@ VRAR_API int vrar_set_rd_chunks(int C);
 VRAR_API int vrar_get_rd_chunks(void);
 
 /* Whether ONESHOT / TWOSTAGE / TWOSTAGE_WRITE run the start and end flag
- * barriers of [CAR] (default 1 = yes). Inside one launch on one device the
- * kernel boundary already orders the calls, so 0 drops them; the 2-stage mid
- * barrier always runs because the all-gather reads other ranks' results. */
+ * barriers of [CAR] (default 0 = no). Across devices they keep a rank from
+ * reading a peer's buffer before the peer has entered the call, and from
+ * returning while a peer still reads its buffer. Here every virtual rank runs
+ * in one launch on one stream, so the launch boundaries already give both
+ * guarantees and the barriers only add latency; 1 runs them anyway (same
+ * results). The 2-stage mid barrier always runs: its all-gather reads other
+ * ranks' partial results. */
 VRAR_API int vrar_set_edge_sync(int on);
 VRAR_API int vrar_get_edge_sync(void);
 

@@ -101,7 +101,7 @@ def test_valid_call_without_device_reports_cuda_error():
 
 
 def test_settings_round_trip_and_ranges():
-    assert vrar.get_group_size() == 8 and vrar.get_rd_chunks() == 4 and vrar.get_edge_sync()
+    assert vrar.get_group_size() == 8 and vrar.get_rd_chunks() == 4 and not vrar.get_edge_sync()
     for bad in (0, 33):
         with pytest.raises(vrar.VrarError):
             vrar.set_group_size(bad)
@@ -114,9 +114,9 @@ def test_settings_round_trip_and_ranges():
     vrar.set_spin_timeout_ns(5_000_000)
     assert vrar.get_spin_timeout_ns() == 5_000_000
     vrar.set_spin_timeout_ns(t)
-    vrar.set_edge_sync(False)
-    assert not vrar.get_edge_sync()
     vrar.set_edge_sync(True)
+    assert vrar.get_edge_sync()
+    vrar.set_edge_sync(False)
 
 
 def test_selector_is_defined_for_every_shape():

@@ -32,7 +32,7 @@ def _defaults():
     if vrar is not None:
         vrar.set_group_size(8)
         vrar.set_rd_chunks(4)
-        vrar.set_edge_sync(True)
+        vrar.set_edge_sync(False)
         vrar.set_spin_timeout_ns(2_000_000_000)
         vrar.debug_set_fault_mask(0)
 
@@ -41,7 +41,7 @@ def _dev(xs_np, dtype):
     return [from_np(x, dtype).cuda() for x in xs_np]
 
 
-def run(algo, xs_np, dtype, L=8, C=4, edge=True):
+def run(algo, xs_np, dtype, L=8, C=4, edge=False):
     vrar.set_group_size(L)
     vrar.set_rd_chunks(C)
     vrar.set_edge_sync(edge)
@@ -180,11 +180,13 @@ def test_config_p8_rd_1000_calls_reuse_flags():
     assert rc == 0, info
 
 
-def test_cuda_graph_replay_reuses_flags():
+@pytest.mark.parametrize("edge", [False, True])
+def test_cuda_graph_replay_reuses_flags(edge):
     n = 131_072
     xs = gen(8, n, "bf16", synth.normal(0.0, 1.0), seed=4)
     d_in = _dev(xs, "bf16")
-    for algo in ("rd", "twostage", "oneshot", "twostage_write"):
+    vrar.set_edge_sync(edge)
+    for algo in ("rd", "twostage", "oneshot", "twostage_write", "hier"):
         outs = [torch.empty_like(t) for t in d_in]
         want = oracle.allreduce(algo, xs, "bf16")
         s = torch.cuda.Stream()
@@ -241,6 +243,53 @@ def test_config_p8_prefill_sampled():
 
 
 # ---- protocol properties ----------------------------------------------------------------------
+
+@pytest.mark.parametrize("algo", ["oneshot", "twostage", "twostage_write", "rd", "hier"])
+def test_inputs_written_by_the_previous_kernel(algo):
+    """Calls launch with programmatic dependent launch; a kernel that writes the
+    inputs right before the call (no host sync in between) must be waited for.
+    Integer inputs: after k rounds of `x += 1` on every rank the sum grows by k*P."""
+    P, n = 8, 300_001
+    xs = gen(P, n, "bf16", synth.INT8, seed=21)
+    base = np.stack([oracle.to_float(x, "bf16") for x in xs]).astype(np.int64).sum(axis=0)
+    d_in = _dev(xs, "bf16")
+    outs = [torch.empty_like(t) for t in d_in]
+    vrar.set_group_size(4)
+    for k in range(1, 6):
+        for t in d_in:
+            t.add_(1.0)
+        vrar.all_reduce(d_in, outs, algo=algo)
+        got = oracle.to_float(to_np(outs[3]), "bf16")
+        assert (got == base + k * P).all(), f"{algo} round {k}"
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for t in d_in:
+            t.add_(1.0)
+        vrar.all_reduce(d_in, outs, algo=algo)
+    for k in range(6, 11):
+        g.replay()
+        torch.cuda.synchronize()
+        got = oracle.to_float(to_np(outs[5]), "bf16")
+        assert (got == base + k * P).all(), f"{algo} graph round {k}"
+    rc, info = vrar.query_status()
+    assert rc == 0, info
+
+
+def test_chained_calls_read_the_previous_calls_output():
+    """out1 = allreduce(x); out2 = allreduce(out1) back to back: the second
+    kernel reads what the first wrote (P * sum for integer inputs)."""
+    P, n = 4, 200_003
+    xs = gen(P, n, "fp32", synth.INT8, seed=22)
+    base = np.stack(xs).astype(np.int64).sum(axis=0)
+    d_in = _dev(xs, "fp32")
+    mid = [torch.empty_like(t) for t in d_in]
+    out = [torch.empty_like(t) for t in d_in]
+    for a1 in ("oneshot", "twostage_write", "rd", "twostage"):
+        for a2 in ("oneshot", "twostage", "rd", "twostage_write"):
+            vrar.all_reduce(d_in, mid, algo=a1)
+            vrar.all_reduce(mid, out, algo=a2)
+            assert (to_np(out[P - 1]).astype(np.int64) == P * base).all(), (a1, a2)
+
 
 def test_chunk_count_and_edge_sync_do_not_change_results():
     xs = gen(8, 50_001, "bf16", synth.normal(0.0, 1.0), seed=11)
