@@ -25,7 +25,8 @@ if not os.path.exists(LIB_PATH):
                       "(python collective_all_reduce_virtual_b200/build.py)")
 _lib = ctypes.CDLL(LIB_PATH)
 
-OK, EINVAL, ENOTSUP, ENOMEM, ECUDA, ETIMEDOUT = 0, -1, -2, -3, -4, -5
+OK, EINVAL, ENOTSUP, ENOMEM, ECUDA, ETIMEDOUT, ETOOBIG = 0, -1, -2, -3, -4, -5, -6
+NOALLOC_SCRATCH_BYTES = 16 << 20
 MAX_RANKS = 32
 
 DTYPES = {torch.bfloat16: 0, torch.float32: 1}
@@ -53,6 +54,7 @@ SIGNATURES = {
     "vrar_workspace_bytes": ([_i, _sz, _i, _i], _sz),
     "vrar_reset": ([], _i),
     "vrar_debug_set_fault_mask": ([_u32], _i),
+    "vrar_allreduce_rd_noalloc": ([_pp, _pp, _i, _sz, _i, _vp], _i),
     "vrar_strerror": ([_i], ctypes.c_char_p),
     "vrar_version": ([], _i),
 }

@@ -495,6 +495,7 @@ const char* vrar_strerror(int code) {
     case VRAR_ENOMEM: return "workspace allocation failed";
     case VRAR_ECUDA: return "CUDA runtime error";
     case VRAR_ETIMEDOUT: return "a device wait timed out";
+    case VRAR_ETOOBIG: return "request exceeds the fixed scratch of the allocation-free entry point";
     default: return "unknown error";
   }
 }
@@ -502,3 +503,90 @@ const char* vrar_strerror(int code) {
 int vrar_version(void) { return VRAR_VERSION; }
 
 }  // extern "C"
+
+// ---- allocation-free entry point -----------------------------------------------------------
+// vrar_allreduce_rd_noalloc runs the k_rd kernel on a fixed array instead of
+// the allocated workspace: 256 bytes of control words (ticket, status) and
+// then the payload slots. Host code must not pass g_noalloc_scratch itself to
+// a kernel (in host code the name is a host-side stand-in, not a device
+// address); the device address comes from cudaGetSymbolAddress, looked up
+// once per device with that device current.
+
+namespace vrar {
+namespace {
+
+constexpr size_t kNoAllocBytes = VRAR_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kNoAllocCtrlBytes = 256;
+static_assert(kCtrlWords * sizeof(uint32_t) <= kNoAllocCtrlBytes, "control words must fit");
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+struct NoAllocDevice {
+  unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
+  int sms = 0;
+};
+
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc[kMaxDevices];
+
+// Once per device, with that device current: look up the array's device
+// address, zero it (so no payload word or ticket starts with a value a call
+// could take for its own), and read the SM count for grid sizing.
+int noalloc_setup(int dev, NoAllocDevice** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc[dev];
+  if (!d.base) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e);
+    if (cudaMemset(p, 0, kNoAllocBytes) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return cuda_fail(cudaErrorUnknown);
+    d.sms = sms;
+    d.base = static_cast<unsigned char*>(p);
+  }
+  *out = &d;
+  return VRAR_OK;
+}
+
+}  // namespace
+}  // namespace vrar
+
+extern "C" int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* const rank_out[], int P, size_t n,
+                                         vrar_dtype_t dtype, vrar_stream_t stream) {
+  int rc = check_buffers(rank_in, rank_out, P, n, n, dtype);
+  if (rc != VRAR_OK) return rc;
+  if ((rc = check_shape(VRAR_ALGO_RD, P, 1)) != VRAR_OK) return rc;
+  const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
+  const size_t slots = ll_bytes_for(VRAR_ALGO_RD, P, n, dtype, 1);
+  if (static_cast<size_t>(items) > kNoAllocBytes || slots > kNoAllocBytes - kNoAllocCtrlBytes) return VRAR_ETOOBIG;
+  if (n == 0) return VRAR_OK;
+
+  int dev = 0;
+  if ((rc = current_device(&dev)) != VRAR_OK) return rc;
+  NoAllocDevice* d = nullptr;
+  if ((rc = noalloc_setup(dev, &d)) != VRAR_OK) return rc;
+
+  const int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
+  KernelFn fn = dtype == VRAR_BF16 ? pick_kernel<Bf16T>(VRAR_ALGO_RD, C) : pick_kernel<F32T>(VRAR_ALGO_RD, C);
+  KArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int p = 0; p < P; ++p) {
+    a.ptr.in[p] = rank_in[p];
+    a.ptr.out[p] = rank_out[p];
+  }
+  a.n = static_cast<int64_t>(n);
+  a.items = items;
+  a.P = P;
+  a.L = 1;
+  a.steps = ilog2(P);
+  a.chunks = C;
+  a.fault_mask = 0;
+  a.timeout_ns = g_set.timeout_ns.load();
+  a.ctrl = reinterpret_cast<uint32_t*>(d->base);
+  a.sig = nullptr;  // recursive doubling uses no barrier rows
+  a.ll = reinterpret_cast<uint64_t*>(d->base + kNoAllocCtrlBytes);
+  a.B = blocks_per_rank((a.items + C - 1) / C, P, resident_ctas(fn, dev, d->sms));
+  return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -94,7 +94,8 @@ enum {
                             divide P or P/L not 2^k) */
     VRAR_ENOMEM = -3,    /* workspace allocation failed */
     VRAR_ECUDA = -4,     /* a CUDA runtime call failed (no device, launch error, ...) */
-    VRAR_ETIMEDOUT = -5  /* a device wait hit its time limit (reported by vrar_query_status) */
+    VRAR_ETIMEDOUT = -5, /* a device wait hit its time limit (reported by vrar_query_status) */
+    VRAR_ETOOBIG = -6    /* request larger than the fixed scratch of vrar_allreduce_rd_noalloc */
 };
 
 /*
@@ -193,6 +194,39 @@ VRAR_API int vrar_reset(void);
  * of the following calls (until set back to 0), so that their peers' waits
  * run out of time and report VRAR_ETIMEDOUT instead of hanging. */
 VRAR_API int vrar_debug_set_fault_mask(uint32_t mask);
+
+/*
+ * Allocation-free recursive-doubling all-reduce. The sources have no
+ * counterpart of this call; it exists for callers that cannot let a library
+ * allocate device memory: a serving process whose own allocator has already
+ * claimed nearly all of the GPU's memory (a KV-cache pool, say) and must not
+ * have memory taken behind its back, or code that must not block on the
+ * device-wide synchronisation that cudaMalloc / cudaFree can imply.
+ *
+ * Same arguments, rules and results as vrar_allreduce(..., VRAR_ALGO_RD, ...)
+ * (bit for bit), but it never allocates: its payload slots and control words
+ * live in one fixed array of VRAR_NOALLOC_SCRATCH_BYTES compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits. It calls no cudaMalloc, no cudaFree and no allocating library routine.
+ *  - Limit: P must be a power of two and
+ *      256 + P * log2(P) * ceil(n / e) * 32 <= VRAR_NOALLOC_SCRATCH_BYTES,
+ *    e = 8 for bf16, 4 for fp32 (for P = 8 and bf16: n <= 174,760). Larger
+ *    requests return VRAR_ETOOBIG before anything is queued.
+ *  - The first call on a device sets that device up: it looks up the array's
+ *    device address (cudaGetSymbolAddress) and zeroes it, which waits for the
+ *    device. Make that first call before any stream capture.
+ *  - All calls on a device share the one array, and it keeps the last call's
+ *    contents; nothing has to be cleared between calls, because every word a
+ *    call waits for carries that call's sequence number. Calls that overlap on
+ *    the GPU (on different streams, or from several host threads) race on the
+ *    array and give wrong results: keep them ordered on one stream.
+ *  - Device waits are bounded as in every other call, but a wait that runs out
+ *    of time is not reported anywhere the host can read (vrar_query_status
+ *    covers the allocated workspace only).
+ */
+#define VRAR_NOALLOC_SCRATCH_BYTES (16u << 20)
+VRAR_API int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* const rank_out[], int P, size_t n,
+                                       vrar_dtype_t dtype, vrar_stream_t stream);
 
 /* Static description of a return code. */
 VRAR_API const char* vrar_strerror(int code);

@@ -98,6 +98,20 @@ def test_valid_call_without_device_reports_cuda_error():
     assert call_ar(_ptrs(IN, 2), _ptrs(OUT, 2), 2, 64) == vrar.ECUDA
     # adjacent, non-overlapping ranges pass the overlap check
     assert call_ar(vrar.ptr_array([IN, IN + 128]), _ptrs(OUT, 2), 2, 64) == vrar.ECUDA
+    # largest request the fixed scratch holds at P = 8, bf16: passes the size check
+    assert L.vrar_allreduce_rd_noalloc(_ptrs(IN, 8), _ptrs(OUT, 8), 8, 174_760, 0, None) == vrar.ECUDA
+
+
+def test_noalloc_rejects_requests_beyond_its_fixed_scratch():
+    """The allocation-free entry point refuses, on the host, any request whose
+    payload slots would not fit its fixed array (fake pointers: nothing runs)."""
+    f = L.vrar_allreduce_rd_noalloc
+    assert f(_ptrs(IN, 8), _ptrs(OUT, 8), 8, 174_760 + 8, 0, None) == vrar.ETOOBIG
+    # 2^24 fp32 per rank at P = 2: 256 MiB of slots (buffers 1 GiB apart, no overlap)
+    assert f(_ptrs(IN, 2, 1 << 30), _ptrs(OUT, 2, 1 << 30), 2, 1 << 24, 1, None) == vrar.ETOOBIG
+    assert f(_ptrs(IN, 3), _ptrs(OUT, 3), 3, 64, 0, None) == vrar.ENOTSUP
+    assert f(_ptrs(IN, 8), _ptrs(OUT, 8), 8, 0, 0, None) == vrar.OK
+    assert "fixed scratch" in vrar.strerror(vrar.ETOOBIG)
 
 
 def test_settings_round_trip_and_ranges():
