@@ -288,6 +288,27 @@ __device__ __forceinline__ uint4 reduce_item(const RankPtrs& rp, int first, int 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// L2 prefetch hint for [p, p + bytes) (16-byte aligned, bytes a multiple of 16).
+// Kernels issue these for their first inputs between pdl_trigger() and
+// pdl_wait(), i.e. while the previous call may still be running: a prefetch
+// returns no data to the thread, and L2 is the point of coherence of the
+// device, so a line fetched early is updated by any later write to it and no
+// thread can see a stale value. It only moves DRAM latency off the critical
+// path of back-to-back calls.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Prefetch items [first, first + count) of a rank vector of n elements,
+// clipped to the items that lie wholly inside the vector.
+template <class D>
+__device__ __forceinline__ void prefetch_items(const void* base, int64_t first, int64_t count, int64_t n) {
+  const int64_t full = n / D::VE;
+  const int64_t last = first + count < full ? first + count : full;
+  if (last > first)
+    prefetch_l2(static_cast<const char*>(base) + first * 16, static_cast<uint32_t>((last - first) * 16));
+}
+
 // ---- per-call sequence number [NVRAR "Sequence-Number Synchronization"] ------------------
 // One 64-bit ticket per device: every CTA of a call adds 1 (a relaxed atomic:
 // the ticket is the only location involved, and its modification order

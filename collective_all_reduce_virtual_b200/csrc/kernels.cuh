@@ -29,9 +29,12 @@ __device__ __forceinline__ int64_t lo_of(int64_t part, int64_t piece, int64_t to
 // time, so all but the first read of each line hit L2.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_oneshot(const KArgs a) {
-  pdl_wait();
   pdl_trigger();
   Cta c = cta_coords(a);
+  // Rank r's CTAs prefetch input r only: all P ranks read the same items.
+  if (threadIdx.x == 0)
+    prefetch_items<D>(a.ptr.in[c.r], static_cast<int64_t>(c.b) * kThreads, kThreads, a.n);
+  pdl_wait();
   if (a.edge_sync) {
     cta_publish_flag(c, cta_take_ticket(a));
     if (!block_barrier(a, c, kPhStart)) return;
@@ -48,9 +51,15 @@ __global__ void __launch_bounds__(kThreads) k_oneshot(const KArgs a) {
 // barrier. Stage 2: rank r copies every other slice s out of out[s].
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_twostage(const KArgs a) {
-  pdl_wait();
   pdl_trigger();
   Cta c = cta_coords(a);
+  {
+    const int64_t piece = (a.items + a.P - 1) / a.P;
+    const int64_t first = lo_of(c.r, piece, a.items) + static_cast<int64_t>(c.b) * kThreads;
+    const int64_t count = min(static_cast<int64_t>(kThreads), lo_of(c.r + 1, piece, a.items) - first);
+    if (threadIdx.x < a.P) prefetch_items<D>(a.ptr.in[threadIdx.x], first, count, a.n);
+  }
+  pdl_wait();
   const unsigned long long ticket = cta_take_ticket(a);
   if (a.edge_sync) {
     cta_publish_flag(c, ticket);
@@ -94,9 +103,15 @@ __global__ void __launch_bounds__(kThreads) k_twostage(const KArgs a) {
 // the end barrier's flags.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
-  pdl_wait();
   pdl_trigger();
   Cta c = cta_coords(a);
+  {
+    const int64_t piece = (a.items + a.P - 1) / a.P;
+    const int64_t first = lo_of(c.r, piece, a.items) + static_cast<int64_t>(c.b) * kThreads;
+    const int64_t count = min(static_cast<int64_t>(kThreads), lo_of(c.r + 1, piece, a.items) - first);
+    if (threadIdx.x < a.P) prefetch_items<D>(a.ptr.in[threadIdx.x], first, count, a.n);
+  }
+  pdl_wait();
   if (a.edge_sync) {
     cta_publish_flag(c, cta_take_ticket(a));
     if (!block_barrier(a, c, kPhStart)) return;
@@ -165,13 +180,18 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
 
 template <class D, int C>
 __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
-  pdl_wait();
   pdl_trigger();
   Cta c = cta_coords(a);
-  const unsigned long long ticket = cta_take_ticket(a);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
   const int64_t per_chunk = (a.items + C - 1) / C;
+  if (threadIdx.x < C) {
+    const int64_t first = threadIdx.x * per_chunk + static_cast<int64_t>(c.b) * kThreads;
+    const int64_t count = min(static_cast<int64_t>(kThreads), (threadIdx.x + 1) * per_chunk - first);
+    prefetch_items<D>(a.ptr.in[c.r], first, count, a.n);
+  }
+  pdl_wait();
+  const unsigned long long ticket = cta_take_ticket(a);
   bool ok = true;
   // The trip count is the same for every thread of the CTA (the flag is
   // published inside the first trip, after that trip's input loads issue).
@@ -206,16 +226,22 @@ __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
 // L ranks of group g. Slices are cut into C chunks as in k_rd.
 template <class D, int C>
 __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
-  pdl_wait();
   pdl_trigger();
   Cta c = cta_coords(a);
-  const unsigned long long ticket = cta_take_ticket(a);
   const int L = a.L, g = c.r / L, l = c.r % L;
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
   const int64_t piece = (a.items + L - 1) / L;
   const int64_t lo = lo_of(l, piece, a.items), len = lo_of(l + 1, piece, a.items) - lo;
   const int64_t per_chunk = (len + C - 1) / C;
+  if (threadIdx.x < L * C) {  // input rank g*L + (tid / C), chunk tid % C
+    const int k = threadIdx.x % C;
+    const int64_t first = k * per_chunk + static_cast<int64_t>(c.b) * kThreads;
+    const int64_t count = min(static_cast<int64_t>(kThreads), min((k + 1) * per_chunk, len) - first);
+    prefetch_items<D>(a.ptr.in[g * L + threadIdx.x / C], lo + first, count, a.n);
+  }
+  pdl_wait();
+  const unsigned long long ticket = cta_take_ticket(a);
   bool ok = true;
   for (int64_t base = 0; base < per_chunk; base += stride) {  // same trip count in the whole CTA
     const int64_t j = base + t0;
@@ -250,12 +276,17 @@ __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
 // every slice starts on a 16-byte boundary), element path otherwise.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_reduce_scatter(const KArgs a) {
-  pdl_wait();
   pdl_trigger();
   const int r = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(b) * kThreads + threadIdx.x;
   const int64_t m = a.n / a.P;
+  if (m % D::VE == 0 && threadIdx.x < a.P) {
+    const int64_t mi = m / D::VE, first = static_cast<int64_t>(b) * kThreads;
+    const int64_t count = min(static_cast<int64_t>(kThreads), mi - first);
+    prefetch_items<D>(a.ptr.in[threadIdx.x], r * mi + first, count, a.n);
+  }
+  pdl_wait();
   if (m % D::VE == 0) {
     const int64_t mi = m / D::VE;
     for (int64_t j = t0; j < mi; j += stride)
@@ -275,12 +306,14 @@ __global__ void __launch_bounds__(kThreads) k_reduce_scatter(const KArgs a) {
 // reads its n/P elements once and streams them to offset s*m of all P outputs.
 template <class D>
 __global__ void __launch_bounds__(kThreads) k_all_gather(const KArgs a) {
-  pdl_wait();
   pdl_trigger();
   const int s = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(b) * kThreads + threadIdx.x;
   const int64_t m = a.n / a.P;
+  if (m % D::VE == 0 && threadIdx.x == 0)
+    prefetch_items<D>(a.ptr.in[s], static_cast<int64_t>(b) * kThreads, kThreads, m);
+  pdl_wait();
   if (m % D::VE == 0) {
     const int64_t mi = m / D::VE;
     for (int64_t j = t0; j < mi; j += stride) {

@@ -171,6 +171,13 @@ size_t ll_bytes_for(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L) {
 
 using KernelFn = void (*)(KArgs);
 
+// Upper bound on CTAs per SM a call may use (0 = as many as fit). Leaving
+// room lets the next call's CTAs become resident, and start their L2
+// prefetches, while this call is still running.
+#ifndef VRAR_CTAS_PER_SM
+#define VRAR_CTAS_PER_SM 0
+#endif
+
 // CTAs resident per SM for a kernel (cached per kernel and device).
 int resident_ctas(KernelFn fn, int dev, int sms) {
   struct Entry {
@@ -189,6 +196,7 @@ int resident_ctas(KernelFn fn, int dev, int sms) {
     cudaGetLastError();
     occ = 1;
   }
+  if (VRAR_CTAS_PER_SM > 0 && occ > VRAR_CTAS_PER_SM) occ = VRAR_CTAS_PER_SM;
   if (used < 256) cache[used++] = {fn, dev, occ};
   return occ * sms;
 }
@@ -275,10 +283,16 @@ int env_algo() {
   return v;
 }
 
+// Per-size choice, from CUDA-graph timings of back-to-back calls on a B200
+// (the benchmark's per-algorithm sweep): one-shot is one pass with no
+// exchange and wins while its P-fold re-reads still come from L2 quickly
+// (P <= 8 up to 256 KiB per rank); above that, or with more ranks, the write
+// mode's minimum traffic wins. Recursive doubling and the hierarchical
+// algorithm move 2x the data as payload words and never win on one device.
 int select_algo(int P, size_t n, vrar_dtype_t dt) {
   const size_t bytes = n * elem_size(dt);
   if (P <= 1) return VRAR_ALGO_ONESHOT;
-  if (bytes <= (256u << 10)) return VRAR_ALGO_ONESHOT;
+  if (P <= 8 && bytes <= (256u << 10)) return VRAR_ALGO_ONESHOT;
   return VRAR_ALGO_TWOSTAGE_WRITE;
 }
 
