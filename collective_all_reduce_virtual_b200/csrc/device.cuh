@@ -43,7 +43,7 @@ enum Ctrl : int {
   kCtrlWords = 16
 };
 
-enum Phase : uint32_t { kPhStart = 1, kPhMid = 2, kPhEnd = 3, kPhPayload = 4 };
+enum Phase : uint32_t { kPhStart = 1, kPhMid = 2, kPhEnd = 3, kPhPayload = 4, kPhCopy = 5 };
 constexpr uint32_t kErrTimeout = 1;
 
 struct RankPtrs {
@@ -62,6 +62,7 @@ struct KArgs {
   int steps;         // recursive-doubling steps (log2 of the ranks doubled over)
   int chunks;        // payload pieces in flight per thread and step
   int edge_sync;     // run start/end barriers
+  int stages;        // shared-memory pipeline depth (staged kernels)
   uint32_t fault_mask;
   uint64_t timeout_ns;
   uint32_t* ctrl;
@@ -141,6 +142,55 @@ __device__ __forceinline__ void st_payload2(uint64_t* p, uint64_t a, uint64_t b)
 
 __device__ __forceinline__ void ld_payload2(const uint64_t* p, uint64_t& a, uint64_t& b) {
   asm volatile("ld.relaxed.gpu.global.v2.u64 {%0,%1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+
+// ---- shared-memory pipelines: mbarriers and bulk copies (no multicast) -------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make mbarrier initialisation visible to the async proxy (the bulk copies).
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// One bulk copy global -> this CTA's shared memory, completing `bytes` of the
+// barrier's transaction count. 16-byte aligned addresses, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+  return v;
 }
 
 // ---- element types ----------------------------------------------------------------

@@ -28,7 +28,7 @@ __device__ __forceinline__ int64_t lo_of(int64_t part, int64_t piece, int64_t to
 // barriers. The P CTAs with the same b read the same items at about the same
 // time, so all but the first read of each line hit L2.
 template <class D>
-__global__ void __launch_bounds__(kThreads) k_oneshot(const KArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) k_oneshot(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
   // Rank r's CTAs prefetch input r only: all P ranks read the same items.
@@ -125,6 +125,141 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
       const int p = (c.r + j) % a.P;
       store_item<D, true>(a.ptr.out[p], it, a.n, v);
     }
+  }
+  if (a.edge_sync) {
+    __threadfence();
+    block_barrier(a, c, kPhEnd);
+  }
+}
+
+// 2-stage write mode, staged through shared memory with bulk copies. Same
+// result and same work split by rank as k_twostage_write: rank r reduces slice
+// r and streams it to all P outputs. The slice is cut into tiles of
+// kStageItems items; CTA b of rank r takes tiles b, b+B, b+2B, ... A producer
+// (lane 0 of warp 0) keeps up to `stages` tiles in flight: per tile, one bulk
+// copy per input rank (2 KiB each) into a shared-memory stage, completing an
+// mbarrier transaction count. Consumer warps (one thread per item) sum the P
+// copies of their item from shared memory in ascending rank order, round once,
+// and store the result to the P outputs, then free the stage for the producer.
+// Loads of later tiles thus overlap stores of earlier ones without holding P
+// vectors per thread in registers. A ragged last item (n not a multiple of the
+// item size) is reduced from global memory by one thread.
+
+// Bounded mbarrier wait. Gives up when the time limit passes (recording a
+// timeout) or when another thread of the CTA has given up (abort flag).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const KArgs& a, const Cta& c,
+                                          volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > a.timeout_ns) {
+        *abort_flag = 1;
+        report_timeout(a, c, kPhCopy);
+        return false;
+      }
+    }
+  }
+}
+
+template <class D, int kStageItems>
+__global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(const KArgs a) {
+  constexpr uint32_t kStageTileBytes = kStageItems * 16;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_abort;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // stages x 8 bytes, then stages x 8 bytes
+  uint64_t* empty = full + a.stages;
+  unsigned char* stage0 = smem + 128;
+  const int S = a.stages;
+  const size_t stage_bytes = static_cast<size_t>(a.P) * kStageTileBytes;
+
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const int64_t full_items = a.n / D::VE;  // items wholly inside the vector
+  const int64_t piece = (a.items + a.P - 1) / a.P;
+  const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
+  const int64_t hi_full = hi < full_items ? hi : full_items;
+  const int64_t rank_tiles = hi_full > lo ? (hi_full - lo + kStageItems - 1) / kStageItems : 0;
+  const int64_t ntile = rank_tiles > c.b ? (rank_tiles - c.b + a.B - 1) / a.B : 0;
+  auto tile_base = [&](int64_t k) { return lo + (c.b + k * a.B) * kStageItems; };
+
+  if (threadIdx.x < a.P) {  // warm L2 with the first tiles while the previous call drains
+    for (int64_t k = 0; k < ntile && k < S; ++k) {
+      const int64_t base = tile_base(k);
+      prefetch_items<D>(a.ptr.in[threadIdx.x], base, hi_full - base < kStageItems ? hi_full - base : kStageItems,
+                        a.n);
+    }
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kStageItems / 32);
+    }
+    s_abort = 0;
+    mbar_init_fence();
+  }
+  __syncthreads();
+  pdl_wait();
+  if (a.edge_sync) {
+    cta_publish_flag(c, cta_take_ticket(a));
+    if (!block_barrier(a, c, kPhStart)) return;  // no copy issued yet
+  }
+  volatile int* abort_flag = &s_abort;
+
+  if (threadIdx.x == 0) {
+    // Producer.
+    int64_t issued = 0;
+    for (int64_t k = 0; k < ntile; ++k) {
+      const int st = static_cast<int>(k % S);
+      if (k >= S && !mbar_wait(&empty[st], static_cast<uint32_t>((k / S) & 1) ^ 1u, a, c, abort_flag)) break;
+      const int64_t base = tile_base(k);
+      const uint32_t bytes =
+          static_cast<uint32_t>((hi_full - base < kStageItems ? hi_full - base : kStageItems) * 16);
+      mbar_arrive_expect_tx(&full[st], bytes * a.P);
+      unsigned char* dst = stage0 + st * stage_bytes;
+      for (int p = 0; p < a.P; ++p)
+        bulk_load(dst + p * kStageTileBytes, static_cast<const unsigned char*>(a.ptr.in[p]) + base * 16, bytes,
+                  &full[st]);
+      issued = k + 1;
+    }
+    if (*abort_flag) {
+      // Let the copies still in flight land before the CTA's shared memory goes away.
+      for (int64_t k = issued > S ? issued - S : 0; k < issued; ++k) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[k % S], static_cast<uint32_t>((k / S) & 1)) &&
+               globaltimer_ns() - t0 < a.timeout_ns) {
+        }
+      }
+    }
+  } else if (threadIdx.x >= 32) {
+    // Consumers: thread i takes item i of every tile.
+    const int ci = threadIdx.x - 32;
+    for (int64_t k = 0; k < ntile; ++k) {
+      const int st = static_cast<int>(k % S);
+      bool ok = mbar_wait(&full[st], static_cast<uint32_t>((k / S) & 1), a, c, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int64_t base = tile_base(k);
+      if (base + ci < hi_full) {
+        const unsigned char* src = stage0 + st * stage_bytes + ci * 16;
+        Acc<D> acc;
+        acc.init(ld_shared_v4(src));
+        for (int p = 1; p < a.P; ++p) acc.add(ld_shared_v4(src + p * kStageTileBytes));
+        const uint4 v = acc.round();
+        for (int j = 0; j < a.P; ++j) {
+          const int q = (c.r + j) % a.P;
+          st_stream(static_cast<typename D::E*>(a.ptr.out[q]) + (base + ci) * D::VE, v);
+        }
+      }
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[st]);
+    }
+  }
+  // Ragged last item, by the slice owner's first CTA.
+  if (threadIdx.x == 32 && c.b == 0 && full_items < a.items && full_items >= lo && full_items < hi) {
+    const uint4 v = reduce_item<D>(a.ptr, 0, a.P, full_items, a.n);
+    for (int p = 0; p < a.P; ++p) store_item<D, true>(a.ptr.out[p], full_items, a.n, v);
   }
   if (a.edge_sync) {
     __threadfence();
@@ -275,7 +410,7 @@ __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
 // Needs no flags. 16-byte path when m is a multiple of the item size (so
 // every slice starts on a 16-byte boundary), element path otherwise.
 template <class D>
-__global__ void __launch_bounds__(kThreads) k_reduce_scatter(const KArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) k_reduce_scatter(const KArgs a) {
   pdl_trigger();
   const int r = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
@@ -305,7 +440,7 @@ __global__ void __launch_bounds__(kThreads) k_reduce_scatter(const KArgs a) {
 // Standalone all-gather [NVRAR phase 3 over one group], push form: rank s
 // reads its n/P elements once and streams them to offset s*m of all P outputs.
 template <class D>
-__global__ void __launch_bounds__(kThreads) k_all_gather(const KArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) k_all_gather(const KArgs a) {
   pdl_trigger();
   const int s = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;

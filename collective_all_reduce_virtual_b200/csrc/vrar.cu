@@ -178,26 +178,56 @@ using KernelFn = void (*)(KArgs);
 #define VRAR_CTAS_PER_SM 0
 #endif
 
-// CTAs resident per SM for a kernel (cached per kernel and device).
-int resident_ctas(KernelFn fn, int dev, int sms) {
+// Raise a kernel's dynamic shared-memory limit on the current device to at
+// least `smem` bytes (never lowers it: an earlier, larger launch may rely on it).
+bool ensure_smem_limit(KernelFn fn, int dev, size_t smem) {
   struct Entry {
     KernelFn fn;
     int dev;
+    size_t limit;
+  };
+  static std::mutex mu;
+  static Entry set[256];
+  static int used = 0;
+  if (smem <= 48 * 1024) return true;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* e = nullptr;
+  for (int i = 0; i < used; ++i)
+    if (set[i].fn == fn && set[i].dev == dev) e = &set[i];
+  if (e && e->limit >= smem) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (e) e->limit = smem;
+  else if (used < 256) set[used++] = {fn, dev, smem};
+  return true;
+}
+
+// CTAs resident per SM for a kernel with `threads` threads and `smem` bytes of
+// dynamic shared memory (cached per kernel, device and smem size); 0 if the
+// kernel cannot be given that much shared memory.
+int resident_ctas(KernelFn fn, int dev, int sms, int threads = kThreads, size_t smem = 0) {
+  struct Entry {
+    KernelFn fn;
+    int dev;
+    size_t smem;
     int occ;
   };
   static std::mutex mu;
-  static Entry cache[256];
+  static Entry cache[512];
   static int used = 0;
+  if (!ensure_smem_limit(fn, dev, smem)) return 0;
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < used; ++i)
-    if (cache[i].fn == fn && cache[i].dev == dev) return cache[i].occ * sms;
+    if (cache[i].fn == fn && cache[i].dev == dev && cache[i].smem == smem) return cache[i].occ * sms;
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, 0) != cudaSuccess || occ < 1) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem) != cudaSuccess || occ < 1) {
     cudaGetLastError();
     occ = 1;
   }
   if (VRAR_CTAS_PER_SM > 0 && occ > VRAR_CTAS_PER_SM) occ = VRAR_CTAS_PER_SM;
-  if (used < 256) cache[used++] = {fn, dev, occ};
+  if (used < 512) cache[used++] = {fn, dev, smem, occ};
   return occ * sms;
 }
 
@@ -243,11 +273,11 @@ bool pdl_enabled() {
   return cached == 1;
 }
 
-int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream) {
+int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream, int threads = kThreads, size_t smem = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -257,6 +287,59 @@ int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream) {
   cudaError_t e = cudaLaunchKernelEx(&cfg, fn, a);
   if (e != cudaSuccess) return cuda_fail(e);
   return VRAR_OK;
+}
+
+// Which write-mode kernel runs: VRAR_WRITE_KERNEL=plain|staged forces one
+// (read once); otherwise write_staged_for() decides by shape.
+int write_kernel_override() {
+  static int cached = -2;
+  if (cached == -2) {
+    const char* s = std::getenv("VRAR_WRITE_KERNEL");
+    cached = !s ? -1 : std::strcmp(s, "plain") == 0 ? 0 : std::strcmp(s, "staged") == 0 ? 1 : -1;
+  }
+  return cached;
+}
+
+// Per-shape choice measured on a B200 (CUDA-graph timings of back-to-back
+// calls, inputs rotated through more than 3x the L2 size): 'O' one-shot,
+// 'P' write mode with the plain kernel, 'S' write mode with the shared-memory
+// staged kernel. Rows: P <= 2, 4, 8, 16, 32; columns: bytes per rank
+// <= 32 KiB, 64 KiB, ..., 8 MiB, and above. One-shot wins small messages at
+// few ranks (a single pass, its P-fold re-reads served by L2); the write mode
+// moves the minimum traffic and wins everywhere else; the staged kernel
+// overlaps tile loads with stores and wins except around 1 MiB per rank and
+// at 32 ranks above 2 MiB.
+constexpr char kChoice[5][10] = {
+    {'O', 'O', 'O', 'O', 'O', 'O', 'O', 'S', 'S', 'S'},  // P <= 2
+    {'O', 'O', 'O', 'O', 'O', 'P', 'S', 'S', 'S', 'S'},  // P <= 4
+    {'O', 'O', 'O', 'O', 'S', 'P', 'S', 'S', 'S', 'S'},  // P <= 8
+    {'S', 'S', 'S', 'S', 'S', 'P', 'P', 'S', 'S', 'S'},  // P <= 16
+    {'S', 'S', 'S', 'S', 'S', 'P', 'S', 'P', 'P', 'P'},  // P <= 32
+};
+
+char shape_choice(int P, size_t bytes) {
+  if (P <= 1) return 'O';
+  const int row = P <= 2 ? 0 : P <= 4 ? 1 : P <= 8 ? 2 : P <= 16 ? 3 : 4;
+  int col = 0;
+  while (col < 9 && bytes > (static_cast<size_t>(32) << 10 << col)) ++col;
+  return kChoice[row][col];
+}
+
+bool write_staged_for(int P, size_t bytes) {
+  const int forced = write_kernel_override();
+  if (forced >= 0) return forced == 1;
+  return shape_choice(P, bytes) != 'P';
+}
+
+constexpr int kWriteTileItems = 64;  // staged write mode: items per tile (1 KiB per input rank)
+
+template <class D>
+KernelFn staged_kernel(int ti) {
+  switch (ti) {
+    case 32: return k_twostage_write_staged<D, 32>;
+    case 64: return k_twostage_write_staged<D, 64>;
+    default: return k_twostage_write_staged<D, 128>;
+  }
 }
 
 const char* algo_name(int a) {
@@ -283,17 +366,11 @@ int env_algo() {
   return v;
 }
 
-// Per-size choice, from CUDA-graph timings of back-to-back calls on a B200
-// (the benchmark's per-algorithm sweep): one-shot is one pass with no
-// exchange and wins while its P-fold re-reads still come from L2 quickly
-// (P <= 8 up to 256 KiB per rank); above that, or with more ranks, the write
-// mode's minimum traffic wins. Recursive doubling and the hierarchical
-// algorithm move 2x the data as payload words and never win on one device.
+// The algorithm VRAR_ALGO_AUTO runs: one-shot or write mode per the measured
+// table above. Recursive doubling and the hierarchical algorithm move 2x the
+// data as payload words and never win on one device.
 int select_algo(int P, size_t n, vrar_dtype_t dt) {
-  const size_t bytes = n * elem_size(dt);
-  if (P <= 1) return VRAR_ALGO_ONESHOT;
-  if (P <= 8 && bytes <= (256u << 10)) return VRAR_ALGO_ONESHOT;
-  return VRAR_ALGO_TWOSTAGE_WRITE;
+  return shape_choice(P, n * elem_size(dt)) == 'O' ? VRAR_ALGO_ONESHOT : VRAR_ALGO_TWOSTAGE_WRITE;
 }
 
 }  // namespace
@@ -358,6 +435,21 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
       break;
     }
     default: break;
+  }
+  if (algo == VRAR_ALGO_TWOSTAGE_WRITE && write_staged_for(P, n * elem_size(dtype))) {
+    const int ti = kWriteTileItems;
+    KernelFn sf = dtype == VRAR_BF16 ? staged_kernel<Bf16T>(ti) : staged_kernel<F32T>(ti);
+    const int64_t tiles = std::max<int64_t>(1, (work + ti - 1) / ti);
+    // About 96 KiB of stages per CTA (two CTAs per SM), 2 to 6 stages; one tile
+    // per CTA where the resident grid allows it (more CTAs beat an even split).
+    const int S = std::max(2, std::min(6, (96 * 1024) / (P * ti * 16)));
+    const size_t smem = 128 + static_cast<size_t>(S) * P * ti * 16;
+    const int resident = resident_ctas(sf, dev, ws->sms, 32 + ti, smem);
+    const int B = static_cast<int>(std::min<int64_t>(tiles, std::max(1, std::min(resident, kMaxCtas) / P)));
+    if (resident < 1) return VRAR_ECUDA;
+    a.stages = S;
+    a.B = B;
+    return launch(sf, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), 32 + ti, smem);
   }
   a.B = blocks_per_rank(work, P, resident_ctas(fn, dev, ws->sms));
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));

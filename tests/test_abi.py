@@ -143,6 +143,19 @@ def test_selector_is_defined_for_every_shape():
                     assert P & (P - 1) == 0
 
 
+def test_selector_table_entries():
+    """A few entries of the measured per-shape table (bytes per rank)."""
+    bf = torch.bfloat16
+    assert vrar.select_algo(1, 1 << 20, bf) == "oneshot"            # a copy
+    assert vrar.select_algo(2, 1 << 20, bf) == "oneshot"            # 2 MiB at 2 ranks
+    assert vrar.select_algo(2, 4 << 20, bf) == "twostage_write"     # 8 MiB at 2 ranks
+    assert vrar.select_algo(8, 65536, bf) == "oneshot"              # 128 KiB at 8 ranks
+    assert vrar.select_algo(8, 524288, bf) == "twostage_write"      # 1 MiB at 8 ranks (the decode shape)
+    assert vrar.select_algo(8, 117440512, bf) == "twostage_write"   # prefill
+    assert vrar.select_algo(32, 16384, bf) == "twostage_write"      # 32 KiB at 32 ranks
+    assert vrar.select_algo(8, 65536, torch.float32) == "oneshot"   # 256 KiB in fp32
+
+
 def test_workspace_bytes():
     # RD at P=8 on 2 MiB of bf16 per rank: 8 ranks x 3 steps x 131072 items x 32 bytes
     assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 8 * 3 * 131072 * 32
