@@ -496,6 +496,49 @@ def run_reference(args):
             "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_selector_sweep(args):
+    """Every algorithm at every (P, bytes per rank) of the selector table, as
+    JSON lines (one per shape). The write-mode kernel is the one this process
+    runs (VRAR_WRITE_KERNEL=plain|staged forces one)."""
+    import collective_all_reduce_virtual_b200 as vrar
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    kernel = os.environ.get("VRAR_WRITE_KERNEL", "auto")
+    for P in (2, 4, 8, 16, 32):
+        for kib in (32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384):
+            spec = dict(WORKLOAD, P=P, n=kib * 512, name=f"P={P} {kib} KiB per rank")
+            wl = Workload(spec, device)
+            row = {"P": P, "kib": kib, "write_kernel": kernel, "auto": vrar.select_algo(P, wl.n, TDT[wl.dt])}
+            steps = 200 if kib <= 4096 else 50
+            algos = ("oneshot", "twostage_write", "twostage", "rd") if kernel != "staged" else ("twostage_write",)
+            for algo in algos:
+                if algo == "rd" and P & (P - 1):
+                    continue
+                row[algo] = round(min(measure_algo(wl, algo, steps, 3) for _ in range(3)) * 1e3, 3)
+            wl.free()
+            torch.cuda.empty_cache()
+            print(json.dumps(row), flush=True)
+
+
+def run_case(spec_text: str):
+    """A few back-to-back calls of one algorithm on one shape (for profilers):
+    'algo,P,KiB[,calls]'. Exits non-zero if the device status is not clean."""
+    import collective_all_reduce_virtual_b200 as vrar
+    parts = spec_text.split(",")
+    algo, P, kib = parts[0], int(parts[1]), int(parts[2])
+    calls = int(parts[3]) if len(parts) > 3 else 6
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = Workload(dict(WORKLOAD, P=P, n=kib * 512, name=spec_text), device)
+    h = torch.cuda.current_stream().cuda_stream
+    for i in range(calls):
+        wl.call(i, algo, h)
+    torch.cuda.synchronize()
+    rc, info = vrar.query_status()
+    print(json.dumps({"case": spec_text, "status": rc, "info": info}))
+    return rc
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -505,7 +548,16 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the per-algorithm table and the sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--case", metavar="ALGO,P,KIB[,CALLS]",
+                    help="run a few calls of one algorithm on one shape and exit (for profilers)")
+    ap.add_argument("--selector-sweep", action="store_true",
+                    help="print per-shape timings of every algorithm (JSON lines) and exit")
     args = ap.parse_args(argv)
+    if args.selector_sweep:
+        run_selector_sweep(args)
+        return
+    if args.case:
+        sys.exit(1 if run_case(args.case) else 0)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     line = run_reference(args) if args.impl == "reference" else run_vrar(args)

@@ -1,0 +1,48 @@
+"""Both write-mode kernels (plain and shared-memory staged) against the oracle.
+
+The per-shape table sends each shape to one of the two kernels, so this test
+forces each in turn (VRAR_WRITE_KERNEL is read once per process, hence the
+child processes) over shapes with ragged tails, up to 32 ranks, both dtypes,
+with and without the start/end barriers.
+"""
+
+import os
+import subprocess
+import sys
+import textwrap
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = textwrap.dedent("""
+    import sys
+    sys.path[:0] = [{root!r}, {tests!r}]
+    import numpy as np
+    import collective_all_reduce_virtual_b200 as vrar
+    import oracle, synth
+    from util import from_np, gen, to_np, bits_of
+    for dtype in ("bf16", "fp32"):
+        for P, n in ((1, 1001), (2, 7), (3, 66_001), (8, 9), (8, 300_007), (16, 70_001), (32, 33_333), (32, 1_000_003)):
+            xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P + n)
+            want = oracle.allreduce("twostage_write", xs, dtype)
+            for edge in (False, True):
+                vrar.set_edge_sync(edge)
+                outs = vrar.all_reduce([from_np(x, dtype).cuda() for x in xs], algo="twostage_write")
+                rc, info = vrar.query_status()
+                assert rc == 0, (rc, info)
+                for p in range(P):
+                    assert np.array_equal(bits_of(to_np(outs[p])), bits_of(want[p])), (dtype, P, n, edge, p)
+    print("ok")
+""")
+
+
+@pytest.mark.parametrize("variant", ["plain", "staged"])
+def test_write_kernel_variant_matches_oracle(variant):
+    env = dict(os.environ, VRAR_WRITE_KERNEL=variant)
+    code = CHILD.format(root=ROOT, tests=os.path.join(ROOT, "tests"))
+    res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0 and "ok" in res.stdout, res.stdout[-2000:] + res.stderr[-4000:]
