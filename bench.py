@@ -417,7 +417,7 @@ def run_vrar(args):
                 vrar.set_group_size(spec["L"])
             w = Workload(spec, device)
             row = {"workload": spec["name"], "P": w.P, "n": w.n, "rotating_sets": w.R,
-                   "auto": vrar.select_algo(w.P, w.n, TDT[w.dt])}
+                   "selected": vrar.select_algo(w.P, w.n, TDT[w.dt])}
             for algo in spec["algos"]:
                 k = spec.get("steps", 200)
                 row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device) / 1e3, peak)
@@ -508,7 +508,7 @@ def run_selector_sweep(args):
         for kib in (32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384):
             spec = dict(WORKLOAD, P=P, n=kib * 512, name=f"P={P} {kib} KiB per rank")
             wl = Workload(spec, device)
-            row = {"P": P, "kib": kib, "write_kernel": kernel, "auto": vrar.select_algo(P, wl.n, TDT[wl.dt])}
+            row = {"P": P, "kib": kib, "write_kernel": kernel, "selected": vrar.select_algo(P, wl.n, TDT[wl.dt])}
             steps = 200 if kib <= 4096 else 50
             algos = ("oneshot", "twostage_write", "twostage", "rd") if kernel != "staged" else ("twostage_write",)
             for algo in algos:
