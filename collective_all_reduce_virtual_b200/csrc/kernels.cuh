@@ -292,6 +292,7 @@ template <class D, int C, bool kHier>
 __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 (&v)[C], const int64_t (&idx)[C],
                                             const bool (&val)[C], int64_t per_rank) {
   const bool mute = (a.fault_mask >> c.r) & 1u;
+  const uint32_t f = c.flag;
   for (int s = 0; s < a.steps; ++s) {
     const int q = rd_partner<kHier>(c.r, s, a.L);
     uint64_t* dst = a.ll + (static_cast<size_t>(q) * a.steps + s) * per_rank * 4;
@@ -299,14 +300,50 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
     if (!mute) {
 #pragma unroll
       for (int k = 0; k < C; ++k)
-        if (val[k]) send_item(dst + idx[k] * 4, v[k], c.flag);
+        if (val[k]) send_item(dst + idx[k] * 4, v[k], f);
+    }
+    // Poll all C slots together (one L2 round trip per attempt, not C), then
+    // re-poll only the items whose four words do not all carry the flag yet.
+    uint64_t w[C][4];
+    uint32_t pending = 0;
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      if (val[k]) {
+        ld_payload2(src + idx[k] * 4, w[k][0], w[k][1]);
+        ld_payload2(src + idx[k] * 4 + 2, w[k][2], w[k][3]);
+        pending |= 1u << k;
+      }
+    }
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+#pragma unroll
+      for (int k = 0; k < C; ++k)
+        if (((pending >> k) & 1u) && (w[k][0] >> 32) == f && (w[k][1] >> 32) == f && (w[k][2] >> 32) == f &&
+            (w[k][3] >> 32) == f)
+          pending &= ~(1u << k);
+      if (!pending) break;
+      if ((it & 15u) == 15u) {
+        if (t0 == 0) t0 = globaltimer_ns();
+        if (ld_relaxed(a.ctrl + kFailEpoch) == f) return false;
+        if (globaltimer_ns() - t0 > a.timeout_ns) {
+          report_timeout(a, c, kPhPayload);
+          return false;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < C; ++k) {
+        if ((pending >> k) & 1u) {
+          ld_payload2(src + idx[k] * 4, w[k][0], w[k][1]);
+          ld_payload2(src + idx[k] * 4 + 2, w[k][2], w[k][3]);
+        }
+      }
     }
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       if (val[k]) {
-        uint4 w;
-        if (!recv_item(src + idx[k] * 4, w, a, c)) return false;
-        v[k] = add_round<D>(v[k], w);
+        const uint4 peer = make_uint4(static_cast<uint32_t>(w[k][0]), static_cast<uint32_t>(w[k][1]),
+                                      static_cast<uint32_t>(w[k][2]), static_cast<uint32_t>(w[k][3]));
+        v[k] = add_round<D>(v[k], peer);
       }
     }
   }

@@ -273,6 +273,20 @@ bool pdl_enabled() {
   return cached == 1;
 }
 
+// Payload pieces each thread keeps in flight in the RD / HIER exchange: at
+// most the configured C, but no more than it takes for the resident grid to
+// cover a rank's `work` items in one round, so that a short message is spread
+// over many threads instead of being stacked C deep on a few. Results do not
+// depend on this choice.
+template <class D>
+int rd_chunks_for(vrar_algo_t algo, int C, int64_t work, int P, int dev, int sms) {
+  for (int c = 1; c < C; ++c) {
+    const int cap = std::max(1, std::min(resident_ctas(pick_kernel<D>(algo, c), dev, sms), kMaxCtas) / P);
+    if ((work + c - 1) / c <= static_cast<int64_t>(cap) * kThreads) return c;
+  }
+  return C;
+}
+
 int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream, int threads = kThreads, size_t smem = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -397,7 +411,13 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   Workspace* ws = nullptr;
   if ((rc = ensure_workspace(dev, ll_bytes_for(algo, P, n, dtype, L), &ws)) != VRAR_OK) return rc;
 
-  const int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
+  int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
+  if (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER) {
+    const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
+    const int64_t work = algo == VRAR_ALGO_RD ? items : (items + L - 1) / L;
+    C = dtype == VRAR_BF16 ? rd_chunks_for<Bf16T>(algo, C, work, P, dev, ws->sms)
+                           : rd_chunks_for<F32T>(algo, C, work, P, dev, ws->sms);
+  }
   KernelFn fn = dtype == VRAR_BF16 ? pick_kernel<Bf16T>(algo, C) : pick_kernel<F32T>(algo, C);
   if (!fn) return VRAR_EINVAL;
 
@@ -674,7 +694,9 @@ extern "C" int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* cons
   NoAllocDevice* d = nullptr;
   if ((rc = noalloc_setup(dev, &d)) != VRAR_OK) return rc;
 
-  const int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
+  int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
+  C = dtype == VRAR_BF16 ? rd_chunks_for<Bf16T>(VRAR_ALGO_RD, C, items, P, dev, d->sms)
+                         : rd_chunks_for<F32T>(VRAR_ALGO_RD, C, items, P, dev, d->sms);
   KernelFn fn = dtype == VRAR_BF16 ? pick_kernel<Bf16T>(VRAR_ALGO_RD, C) : pick_kernel<F32T>(VRAR_ALGO_RD, C);
   KArgs a;
   std::memset(&a, 0, sizeof(a));

@@ -149,9 +149,11 @@ VRAR_API int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype);
 VRAR_API int vrar_set_group_size(int L);
 VRAR_API int vrar_get_group_size(void);
 
-/* Chunk count C of the recursive-doubling exchange (default 4): every thread
- * keeps C payload pieces in flight per step ([NVRAR] "Chunked Non-blocking
- * Communication"). Results do not depend on C. Range 1..8. */
+/* Chunk count C of the recursive-doubling exchange (default 4): the vector is
+ * cut into chunks and every thread keeps up to C payload pieces, one per chunk,
+ * in flight per step ([NVRAR] "Chunked Non-blocking Communication"). A call
+ * uses fewer than C when its grid has threads to spare for a short message.
+ * Results do not depend on C. Range 1..8. */
 VRAR_API int vrar_set_rd_chunks(int C);
 VRAR_API int vrar_get_rd_chunks(void);
 

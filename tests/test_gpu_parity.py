@@ -292,7 +292,9 @@ def test_chained_calls_read_the_previous_calls_output():
 
 
 def test_chunk_count_and_edge_sync_do_not_change_results():
-    xs = gen(8, 50_001, "bf16", synth.normal(0.0, 1.0), seed=11)
+    # Large enough that the grid needs several pieces per thread (a call uses
+    # fewer chunks than configured only when threads are to spare).
+    xs = gen(8, 1_000_003, "bf16", synth.normal(0.0, 1.0), seed=11)
     ref = run("rd", xs, "bf16", C=1)
     for C in range(2, 9):
         assert_bits(run("rd", xs, "bf16", C=C), ref, f"rd C={C}")
