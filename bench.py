@@ -59,7 +59,7 @@ WORKLOAD = dict(name="decode 64x8192 bf16, P=8 virtual ranks (1 MiB per rank), N
 
 SWEEP = (
     [dict(name=f"P=8 sweep {b >> 10} KiB per rank, N(0,1)", P=8, n=b // 2, dtype="bf16", dist="normal:0,1",
-          algos=("oneshot", "twostage", "twostage_write", "rd", "auto")) for b in
+          algos=("oneshot", "twostage", "twostage_write", "rd", "auto"), collectives=("rs", "ag")) for b in
      (128 << 10, 256 << 10, 512 << 10, 1 << 20, 2 << 20)]
     + [dict(name="P=2 ints 128 KiB per rank", P=2, n=65536, dtype="bf16", dist="int8",
             algos=("oneshot", "rd", "auto"))]
@@ -67,7 +67,8 @@ SWEEP = (
             dist="uniform:-1,1", L=8, algos=("hier", "oneshot", "twostage_write", "auto")) for b in
        (256 << 10, 2 << 20)]
     + [dict(name="P=8 prefill 16384x7168 bf16 (224 MiB per rank), N(0,0.02)", P=8, n=16384 * 7168,
-            dtype="bf16", dist="normal:0,0.02", algos=("twostage", "twostage_write", "auto"), steps=20)]
+            dtype="bf16", dist="normal:0,0.02", algos=("twostage", "twostage_write", "auto"), steps=20,
+            collectives=("rs", "ag"))]
 )
 
 # The oracle algorithm the reference arm times: the same summation the GPU
@@ -313,6 +314,44 @@ def measure_algo(wl: Workload, algo: str, steps: int, warmup: int, world=1, devi
     return ms / steps
 
 
+def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1, device=None):
+    """Milliseconds per call of the standalone reduce-scatter ('rs') or
+    all-gather ('ag') on the workload's shape (graph of `steps` calls)."""
+    vrar = wl.vrar
+    lib, P, n = wl.lib, wl.P, wl.n
+    m = n // P
+    small = [[torch.empty(m, dtype=wl.base[0].dtype, device=wl.base[0].device) for _ in range(P)]
+             for _ in range(wl.R)]
+    small_arr = [vrar.ptr_array([t.data_ptr() for t in s]) for s in small]
+
+    def call(i, h):
+        r = i % wl.R
+        if kind == "rs":
+            rc = lib.vrar_reduce_scatter(wl.in_arr[r], small_arr[r], P, n, wl.dtc, h)
+        else:
+            rc = lib.vrar_all_gather(small_arr[r], wl.out_arr[r], P, n, wl.dtc, h)
+        if rc != 0:
+            raise vrar.VrarError(rc, kind)
+
+    call(0, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+
+    def graph(count, offset):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            h = torch.cuda.current_stream().cuda_stream
+            for i in range(count):
+                call(offset + i, h)
+        return g
+
+    gw, gt = graph(warmup, 0), graph(steps, warmup)
+    gw.replay()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(time_graph(gt, world, device), world, device)
+    del gw, gt, small
+    return ms / steps
+
+
 def entry(wl: Workload, t_s: float, peak: float):
     bw = busbw_gbs(wl.P, wl.n, wl.esz, t_s)
     ach = b_min_bytes(wl.P, wl.n, wl.esz) / t_s / 1e9
@@ -421,6 +460,12 @@ def run_vrar(args):
             for algo in spec["algos"]:
                 k = spec.get("steps", 200)
                 row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device) / 1e3, peak)
+            for kind in spec.get("collectives", ()):
+                # RS moves P*n*s in and n*s out; AG n*s in and P*n*s out: (P+1)*n*s either way.
+                t = measure_collective(w, kind, spec.get("steps", 200), 3, world, device) / 1e3
+                ach = (w.P + 1) * w.n * w.esz / t / 1e9
+                row["reduce_scatter" if kind == "rs" else "all_gather"] = {
+                    "us": round(t * 1e6, 3), "hbm_gbs": round(ach, 1), "frac": round(ach / peak, 4)}
             w.free()
             torch.cuda.empty_cache()
             vrar.set_group_size(8)
