@@ -584,6 +584,143 @@ def run_case(spec_text: str):
     return rc
 
 
+def run_spin_stats(args):
+    """Spin statistics of the cross-rank waits over many calls (JSON lines):
+    for each algorithm with waits, `--spin-stats N` calls on the step's
+    workload, as graphs of 1000 calls."""
+    import collective_all_reduce_virtual_b200 as vrar
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = Workload(WORKLOAD, device)
+    per = 1000
+    for algo, edge in (("twostage", False), ("twostage_write", True), ("rd", False)):
+        vrar.set_edge_sync(edge)
+        vrar.set_spin_stats(True)  # before capture: a graph keeps the arguments of its calls
+        wl.call(0, algo, torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        g = wl.graph(algo, per)
+        vrar.get_spin_stats(reset=True)
+        t0 = time.perf_counter()
+        reps = max(1, args.spin_stats // per)
+        for _ in range(reps):
+            g.replay()
+        torch.cuda.synchronize()
+        el = time.perf_counter() - t0
+        vrar.set_spin_stats(False)
+        st = vrar.get_spin_stats(reset=True)
+        rc, info = vrar.query_status()
+        print(json.dumps({"algo": algo, "edge_sync": edge, "calls": reps * per, "seconds": round(el, 2),
+                          "status": rc, **st}), flush=True)
+        del g
+    vrar.set_edge_sync(False)
+
+
+class TboPrefill:
+    """Two micro-batches of a 16k-token prefill through L row-parallel linear
+    layers with P virtual ranks. In each layer rank p multiplies its K/P slice
+    of the micro-batch's activations with its K/P rows of the layer's weight (a
+    plain cuBLAS GEMM through torch: the compute the all-reduce overlaps with),
+    and the P partial outputs are all-reduced; the next layer of that
+    micro-batch reads its slice of the all-reduced output. Random weights; no
+    model is needed."""
+
+    def __init__(self, device, P=8, tokens=8192, hidden=7168, layers=4, seed=0):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        self.P, self.T, self.K, self.H, self.L = P, tokens, hidden, hidden, layers
+        kp = hidden // P
+        self.kp = kp
+        self.x = [torch.randn(tokens, hidden, device=device, dtype=torch.bfloat16, generator=g) for _ in range(2)]
+        self.w = [torch.randn(hidden, hidden, device=device, dtype=torch.bfloat16, generator=g) * 0.02
+                  for _ in range(layers)]
+        self.part = [[torch.empty(tokens, hidden, device=device, dtype=torch.bfloat16) for _ in range(P)]
+                     for _ in range(2)]
+        self.out = [[torch.empty(tokens, hidden, device=device, dtype=torch.bfloat16) for _ in range(P)]
+                    for _ in range(2)]
+
+    def gemm(self, u, layer):
+        kp = self.kp
+        for p in range(self.P):
+            src = self.x[u] if layer == 0 else self.out[u][p]
+            torch.matmul(src[:, p * kp:(p + 1) * kp], self.w[layer][p * kp:(p + 1) * kp, :], out=self.part[u][p])
+
+    def allreduce(self, u, stream=None):
+        import collective_all_reduce_virtual_b200 as vrar
+        vrar.all_reduce(self.part[u], self.out[u], algo="auto", stream=stream)
+
+    def step_sequential(self):
+        for layer in range(self.L):
+            for u in (0, 1):
+                self.gemm(u, layer)
+                self.allreduce(u)
+
+    def step_overlapped(self, comm):
+        """Each all-reduce runs on the comm stream while the other micro-batch
+        computes; a micro-batch's next layer waits for its own all-reduce."""
+        main = torch.cuda.current_stream()
+        done = [None, None]
+        for layer in range(self.L):
+            for u in (0, 1):
+                if done[u] is not None:
+                    main.wait_event(done[u])
+                self.gemm(u, layer)
+                ready = torch.cuda.Event()
+                ready.record(main)
+                comm.wait_event(ready)
+                with torch.cuda.stream(comm):
+                    self.allreduce(u, comm)
+                done[u] = torch.cuda.Event()
+                done[u].record(comm)
+        main.wait_stream(comm)
+
+
+def run_overlap(args):
+    """NEXT-1 shape: sequential vs overlapped 2-micro-batch prefill step."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    m = TboPrefill(device)
+    comm = torch.cuda.Stream()
+
+    def timed(fn, iters):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    import collective_all_reduce_virtual_b200 as vrar
+    it = max(3, args.steps // 20)
+    gemm_flop = m.L * 2 * 2 * m.T * m.K * m.H
+    ar_bytes = m.L * 2 * 2 * m.P * m.T * m.H * 2
+    base = {"workload": f"2 micro-batches x {m.T} tokens, {m.L} layers, hidden {m.H}, row-parallel linear over "
+                        f"P={m.P} virtual ranks (K/P = {m.K // m.P}), bf16, each followed by the all-reduce of "
+                        f"the P partials"}
+    base["gemm_ms"] = timed(lambda: [m.gemm(u, l) for l in range(m.L) for u in (0, 1)], it)
+    base["gemm_tflops"] = gemm_flop / (base["gemm_ms"] * 1e-3) / 1e12
+    base["sequential_ms"] = timed(m.step_sequential, it)
+    rows = []
+    for cap in (0, 148, 96, 64, 48, 32, 24, 16):  # CTA budget of each all-reduce (0 = whole GPU)
+        vrar.set_max_ctas(cap)
+        r = {"max_ctas": cap, "allreduce_ms": timed(lambda: [m.allreduce(u) for _ in range(m.L) for u in (0, 1)], it),
+             "overlapped_ms": timed(lambda: m.step_overlapped(comm), it)}
+        r["allreduce_hbm_gbs"] = ar_bytes / (r["allreduce_ms"] * 1e-3) / 1e9
+        r["speedup_vs_sequential"] = base["sequential_ms"] / r["overlapped_ms"]
+        rows.append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()})
+    vrar.set_max_ctas(0)
+    rc, info = vrar.query_status()
+    base["status"] = rc
+    base["budgets"] = rows
+    best = min(rows, key=lambda r: r["overlapped_ms"])
+    base["best_overlapped_ms"], base["best_max_ctas"] = best["overlapped_ms"], best["max_ctas"]
+    base["saved_ms"] = base["sequential_ms"] - best["overlapped_ms"]
+    print(json.dumps({k: (round(v, 4) if isinstance(v, float) else v) for k, v in base.items()}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -595,6 +732,10 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--case", metavar="ALGO,P,KIB[,CALLS]",
                     help="run a few calls of one algorithm on one shape and exit (for profilers)")
+    ap.add_argument("--spin-stats", type=int, metavar="CALLS", default=0,
+                    help="spin statistics of the waits over CALLS calls per algorithm (JSON lines) and exit")
+    ap.add_argument("--overlap", action="store_true",
+                    help="sequential vs overlapped two-micro-batch prefill step (JSON line) and exit")
     ap.add_argument("--selector-sweep", action="store_true",
                     help="print per-shape timings of every algorithm (JSON lines) and exit")
     args = ap.parse_args(argv)
@@ -603,6 +744,12 @@ def main(argv=None):
         return
     if args.case:
         sys.exit(1 if run_case(args.case) else 0)
+    if args.spin_stats:
+        run_spin_stats(args)
+        return
+    if args.overlap:
+        run_overlap(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     line = run_reference(args) if args.impl == "reference" else run_vrar(args)

@@ -47,12 +47,16 @@ SIGNATURES = {
     "vrar_get_rd_chunks": ([], _i),
     "vrar_set_edge_sync": ([_i], _i),
     "vrar_get_edge_sync": ([], _i),
+    "vrar_set_max_ctas": ([_i], _i),
+    "vrar_get_max_ctas": ([], _i),
     "vrar_set_spin_timeout_ns": ([_u64], _i),
     "vrar_get_spin_timeout_ns": ([], _u64),
     "vrar_query_status": ([_vp, ctypes.POINTER(_u32)], _i),
     "vrar_reserve": ([_sz], _i),
     "vrar_workspace_bytes": ([_i, _sz, _i, _i], _sz),
     "vrar_reset": ([], _i),
+    "vrar_set_spin_stats": ([_i], _i),
+    "vrar_get_spin_stats": ([ctypes.POINTER(_u64), _i], _i),
     "vrar_debug_set_fault_mask": ([_u32], _i),
     "vrar_allreduce_rd_noalloc": ([_pp, _pp, _i, _sz, _i, _vp], _i),
     "vrar_strerror": ([_i], ctypes.c_char_p),
@@ -194,6 +198,15 @@ def get_edge_sync() -> bool:
     return bool(_lib.vrar_get_edge_sync())
 
 
+def set_max_ctas(n: int) -> None:
+    """Cap the CTAs a call launches (0 = as many as fit)."""
+    _check(_lib.vrar_set_max_ctas(n), "vrar_set_max_ctas")
+
+
+def get_max_ctas() -> int:
+    return _lib.vrar_get_max_ctas()
+
+
 def set_spin_timeout_ns(ns: int) -> None:
     _check(_lib.vrar_set_spin_timeout_ns(ns), "vrar_set_spin_timeout_ns")
 
@@ -221,6 +234,20 @@ def reset() -> None:
     _check(_lib.vrar_reset(), "vrar_reset")
 
 
+def set_spin_stats(on: bool) -> None:
+    _check(_lib.vrar_set_spin_stats(1 if on else 0), "vrar_set_spin_stats")
+
+
+SPIN_STAT_KEYS = ("waits", "polls", "max_polls", "long_waits", "timeouts")
+
+
+def get_spin_stats(reset: bool = False) -> dict:
+    """Spin statistics of the current device (waits for the device)."""
+    out = (ctypes.c_uint64 * 5)()
+    _check(_lib.vrar_get_spin_stats(out, 1 if reset else 0), "vrar_get_spin_stats")
+    return dict(zip(SPIN_STAT_KEYS, (int(v) for v in out)))
+
+
 def debug_set_fault_mask(mask: int) -> None:
     _check(_lib.vrar_debug_set_fault_mask(mask), "vrar_debug_set_fault_mask")
 
@@ -235,6 +262,6 @@ def version() -> int:
 
 __all__ = ["all_reduce", "reduce_scatter", "all_gather", "select_algo", "set_group_size",
            "get_group_size", "set_rd_chunks", "get_rd_chunks", "set_edge_sync", "get_edge_sync",
-           "set_spin_timeout_ns", "get_spin_timeout_ns", "query_status", "reserve",
-           "workspace_bytes", "reset", "debug_set_fault_mask", "strerror", "version", "VrarError",
+           "set_max_ctas", "get_max_ctas", "set_spin_timeout_ns", "get_spin_timeout_ns", "query_status", "reserve",
+           "workspace_bytes", "reset", "set_spin_stats", "get_spin_stats", "debug_set_fault_mask", "strerror", "version", "VrarError",
            "ALGOS", "DTYPES", "SIGNATURES", "LIB_PATH", "lib", "ptr_array"]

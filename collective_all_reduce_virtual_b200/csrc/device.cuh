@@ -40,8 +40,13 @@ enum Ctrl : int {
   kStatus = 2,     // sticky error code (0 = none) until the host reads it
   kFailEpoch = 3,  // sequence number of a call in which some wait gave up
   kInfo = 4,       // 4 words: failing call, phase, rank, block
-  kCtrlWords = 16
+  kStats = 16,     // 5 x 64-bit spin statistics (see record_spins), words 16..25
+  kCtrlWords = 32
 };
+
+// Spin statistics counters (64-bit, at ctrl + kStats).
+enum StatIdx : int { kStWaits = 0, kStSpins = 1, kStMax = 2, kStLong = 3, kStTimeouts = 4, kStCount = 5 };
+constexpr uint32_t kLongWaitSpins = 16384;
 
 enum Phase : uint32_t { kPhStart = 1, kPhMid = 2, kPhEnd = 3, kPhPayload = 4, kPhCopy = 5 };
 constexpr uint32_t kErrTimeout = 1;
@@ -68,6 +73,7 @@ struct KArgs {
   uint32_t* ctrl;
   uint32_t* sig;     // kPhases x kSigPhaseWords flag words
   uint64_t* ll;      // payload slots
+  unsigned long long* stats;  // spin statistics, or null when they are off
 };
 
 // ---- PTX wrappers --------------------------------------------------------------
@@ -407,6 +413,29 @@ __device__ __forceinline__ void cta_publish_flag(Cta& c, unsigned long long tick
   c.flag = s_flag;
 }
 
+// Spin statistics of the cross-rank waits, after the temporary instrumentation
+// described in [CAR] "Validation": per wait, the number of polls it took; the
+// counters keep the number of waits, the total and largest poll count, the
+// waits of kLongWaitSpins polls or more, and the waits that hit the time limit
+// (the "safety net"). Off unless the host turned it on (a.stats non-null).
+// The threads of a warp that finish a wait together are combined first, so a
+// warp costs one set of atomics, not 32.
+__device__ __forceinline__ void record_spins(const KArgs& a, uint32_t spins, bool timed_out) {
+  if (!a.stats) return;
+  const unsigned m = __activemask();
+  const uint32_t sum = __reduce_add_sync(m, spins);
+  const uint32_t mx = __reduce_max_sync(m, spins);
+  const uint32_t nlong = __reduce_add_sync(m, spins >= kLongWaitSpins ? 1u : 0u);
+  const uint32_t nto = __reduce_add_sync(m, timed_out ? 1u : 0u);
+  if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(m) - 1)) {
+    atomicAdd(a.stats + kStWaits, static_cast<unsigned long long>(__popc(m)));
+    atomicAdd(a.stats + kStSpins, static_cast<unsigned long long>(sum));
+    atomicMax(a.stats + kStMax, static_cast<unsigned long long>(mx));
+    if (nlong) atomicAdd(a.stats + kStLong, static_cast<unsigned long long>(nlong));
+    if (nto) atomicAdd(a.stats + kStTimeouts, static_cast<unsigned long long>(nto));
+  }
+}
+
 __device__ __noinline__ void report_timeout(const KArgs& a, const Cta& c, uint32_t phase) {
   if (atomicCAS(a.ctrl + kStatus, 0u, kErrTimeout) == 0u) {
     a.ctrl[kInfo + 0] = c.flag;
@@ -421,18 +450,27 @@ __device__ __noinline__ void report_timeout(const KArgs& a, const Cta& c, uint32
 // the time limit passes or another CTA of this call has given up; returns
 // false then. Equality (not >=) keeps the test valid across 32-bit wrap.
 __device__ __forceinline__ bool wait_flag(const uint32_t* p, const KArgs& a, const Cta& c, uint32_t phase) {
-  if (ld_acquire(p) == c.flag) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (ld_acquire(p) == c.flag) return true;
-    if ((it & 63u) == 0u) {
-      if (ld_relaxed(a.ctrl + kFailEpoch) == c.flag) return false;
-      if (globaltimer_ns() - t0 > a.timeout_ns) {
-        report_timeout(a, c, phase);
-        return false;
+  uint32_t polls = 1;
+  bool ok = true;
+  if (ld_acquire(p) != c.flag) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;; ++polls) {
+      if (ld_acquire(p) == c.flag) break;
+      if ((polls & 63u) == 0u) {
+        if (ld_relaxed(a.ctrl + kFailEpoch) == c.flag) {
+          ok = false;
+          break;
+        }
+        if (globaltimer_ns() - t0 > a.timeout_ns) {
+          report_timeout(a, c, phase);
+          record_spins(a, polls, true);
+          return false;
+        }
       }
     }
   }
+  record_spins(a, polls, false);
+  return ok;
 }
 
 // Block barrier across ranks [CAR start_sync / end_sync]: block b of rank r
@@ -463,30 +501,6 @@ __device__ __forceinline__ void send_item(uint64_t* slot, const uint4& v, uint32
   const uint64_t hi = static_cast<uint64_t>(flag) << 32;
   st_payload2(slot, hi | v.x, hi | v.y);
   st_payload2(slot + 2, hi | v.z, hi | v.w);
-}
-
-// Returns false if the wait gave up (time limit, or another CTA gave up).
-__device__ __forceinline__ bool recv_item(const uint64_t* slot, uint4& v, const KArgs& a, const Cta& c) {
-  uint64_t w0, w1, w2, w3;
-  const uint32_t f = c.flag;
-  ld_payload2(slot, w0, w1);
-  ld_payload2(slot + 2, w2, w3);
-  uint64_t t0 = 0;
-  for (uint32_t it = 1; (w0 >> 32) != f || (w1 >> 32) != f || (w2 >> 32) != f || (w3 >> 32) != f; ++it) {
-    if ((w0 >> 32) != f || (w1 >> 32) != f) ld_payload2(slot, w0, w1);
-    if ((w2 >> 32) != f || (w3 >> 32) != f) ld_payload2(slot + 2, w2, w3);
-    if ((it & 63u) == 0u) {
-      if (t0 == 0) t0 = globaltimer_ns();
-      if (ld_relaxed(a.ctrl + kFailEpoch) == f) return false;
-      if (globaltimer_ns() - t0 > a.timeout_ns) {
-        report_timeout(a, c, kPhPayload);
-        return false;
-      }
-    }
-  }
-  v = make_uint4(static_cast<uint32_t>(w0), static_cast<uint32_t>(w1), static_cast<uint32_t>(w2),
-                 static_cast<uint32_t>(w3));
-  return true;
 }
 
 }  // namespace vrar

@@ -145,6 +145,9 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
 // vectors per thread in registers. A ragged last item (n not a multiple of the
 // item size) is reduced from global memory by one thread.
 
+constexpr int kStagedHeader = 512;   // mbarriers of up to kMaxStages stages
+constexpr int kMaxStages = 24;
+
 // Bounded mbarrier wait. Gives up when the time limit passes (recording a
 // timeout) or when another thread of the CTA has given up (abort flag).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const KArgs& a, const Cta& c,
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(cons
   __shared__ int s_abort;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // stages x 8 bytes, then stages x 8 bytes
   uint64_t* empty = full + a.stages;
-  unsigned char* stage0 = smem + 128;
+  unsigned char* stage0 = smem + kStagedHeader;
   const int S = a.stages;
   const size_t stage_bytes = static_cast<size_t>(a.P) * kStageTileBytes;
 
@@ -315,7 +318,8 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
       }
     }
     uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
+    uint32_t it = 0;
+    for (;; ++it) {
 #pragma unroll
       for (int k = 0; k < C; ++k)
         if (((pending >> k) & 1u) && (w[k][0] >> 32) == f && (w[k][1] >> 32) == f && (w[k][2] >> 32) == f &&
@@ -324,9 +328,13 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
       if (!pending) break;
       if ((it & 15u) == 15u) {
         if (t0 == 0) t0 = globaltimer_ns();
-        if (ld_relaxed(a.ctrl + kFailEpoch) == f) return false;
+        if (ld_relaxed(a.ctrl + kFailEpoch) == f) {
+          record_spins(a, it + 1, false);
+          return false;
+        }
         if (globaltimer_ns() - t0 > a.timeout_ns) {
           report_timeout(a, c, kPhPayload);
+          record_spins(a, it + 1, true);
           return false;
         }
       }
@@ -338,6 +346,7 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
         }
       }
     }
+    if (val[0]) record_spins(a, it + 1, false);  // one wait per step (the C pieces are polled together)
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       if (val[k]) {

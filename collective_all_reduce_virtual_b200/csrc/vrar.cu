@@ -25,6 +25,8 @@ struct Settings {
   std::atomic<int> edge_sync{0};
   std::atomic<uint64_t> timeout_ns{2000000000ull};
   std::atomic<uint32_t> fault_mask{0};
+  std::atomic<int> spin_stats{0};
+  std::atomic<int> max_ctas{0};  // grid cap per call, 0 = none
 };
 Settings g_set;
 
@@ -231,6 +233,14 @@ int resident_ctas(KernelFn fn, int dev, int sms, int threads = kThreads, size_t 
   return occ * sms;
 }
 
+// The CTAs one call may use: what fits on the device at once, or fewer if the
+// caller set a budget (vrar_set_max_ctas) to leave SMs to concurrent work.
+int grid_budget(KernelFn fn, int dev, int sms, int threads = kThreads, size_t smem = 0) {
+  const int resident = resident_ctas(fn, dev, sms, threads, smem);
+  const int cap = g_set.max_ctas.load();
+  return (cap > 0 && resident > cap) ? cap : resident;
+}
+
 // CTAs per rank: enough for one item per thread over `work_items` (the items
 // one rank handles), at most what keeps the whole grid resident.
 int blocks_per_rank(int64_t work_items, int P, int max_ctas) {
@@ -281,7 +291,7 @@ bool pdl_enabled() {
 template <class D>
 int rd_chunks_for(vrar_algo_t algo, int C, int64_t work, int P, int dev, int sms) {
   for (int c = 1; c < C; ++c) {
-    const int cap = std::max(1, std::min(resident_ctas(pick_kernel<D>(algo, c), dev, sms), kMaxCtas) / P);
+    const int cap = std::max(1, std::min(grid_budget(pick_kernel<D>(algo, c), dev, sms), kMaxCtas) / P);
     if ((work + c - 1) / c <= static_cast<int64_t>(cap) * kThreads) return c;
   }
   return C;
@@ -438,6 +448,7 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   a.ctrl = ws->ctrl;
   a.sig = ws->sig;
   a.ll = ws->ll;
+  a.stats = g_set.spin_stats.load() ? reinterpret_cast<unsigned long long*>(ws->ctrl + kStats) : nullptr;
 
   int64_t work = a.items;  // items one rank handles in its main loop
   switch (algo) {
@@ -457,21 +468,25 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     default: break;
   }
   if (algo == VRAR_ALGO_TWOSTAGE_WRITE && write_staged_for(P, n * elem_size(dtype))) {
-    const int ti = kWriteTileItems;
+    // Normally 64-item tiles and about 96 KiB of stages per CTA (two CTAs per
+    // SM). When a CTA budget leaves at most one CTA per SM, each CTA must keep
+    // far more bytes in flight to draw its share of memory bandwidth: 128-item
+    // tiles and up to 192 KiB of stages.
+    const int cap_budget = g_set.max_ctas.load();
+    const bool deep = cap_budget > 0 && cap_budget <= ws->sms;
+    const int ti = deep ? 128 : kWriteTileItems;
     KernelFn sf = dtype == VRAR_BF16 ? staged_kernel<Bf16T>(ti) : staged_kernel<F32T>(ti);
     const int64_t tiles = std::max<int64_t>(1, (work + ti - 1) / ti);
-    // About 96 KiB of stages per CTA (two CTAs per SM), 2 to 6 stages; one tile
-    // per CTA where the resident grid allows it (more CTAs beat an even split).
-    const int S = std::max(2, std::min(6, (96 * 1024) / (P * ti * 16)));
-    const size_t smem = 128 + static_cast<size_t>(S) * P * ti * 16;
-    const int resident = resident_ctas(sf, dev, ws->sms, 32 + ti, smem);
+    const int S = std::max(2, std::min(deep ? kMaxStages : 6, ((deep ? 192 : 96) * 1024) / (P * ti * 16)));
+    const size_t smem = kStagedHeader + static_cast<size_t>(S) * P * ti * 16;
+    const int resident = grid_budget(sf, dev, ws->sms, 32 + ti, smem);
     const int B = static_cast<int>(std::min<int64_t>(tiles, std::max(1, std::min(resident, kMaxCtas) / P)));
     if (resident < 1) return VRAR_ECUDA;
     a.stages = S;
     a.B = B;
     return launch(sf, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), 32 + ti, smem);
   }
-  a.B = blocks_per_rank(work, P, resident_ctas(fn, dev, ws->sms));
+  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, ws->sms));
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -497,7 +512,7 @@ int vrar_reduce_scatter(const void* const rank_in[], void* const rank_out[], int
   a.P = P;
   const int64_t m = a.n / P;
   const int64_t work = (m % per_item(dtype) == 0) ? m / per_item(dtype) : m;
-  a.B = blocks_per_rank(work, P, resident_ctas(fn, dev, ws->sms));
+  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, ws->sms));
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -523,7 +538,7 @@ int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, 
   a.P = P;
   const int64_t m = a.n / P;
   const int64_t work = (m % per_item(dtype) == 0) ? m / per_item(dtype) : m;
-  a.B = blocks_per_rank(work, P, resident_ctas(fn, dev, ws->sms));
+  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, ws->sms));
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -605,6 +620,36 @@ int vrar_reset(void) {
   if (w.ll) cudaFree(w.ll);
   if (w.ctrl) cudaFree(w.ctrl);
   w = Workspace();
+  return VRAR_OK;
+}
+
+int vrar_set_max_ctas(int n) {
+  if (n < 0) return VRAR_EINVAL;
+  g_set.max_ctas = n;
+  return VRAR_OK;
+}
+int vrar_get_max_ctas(void) { return g_set.max_ctas.load(); }
+
+int vrar_set_spin_stats(int on) {
+  g_set.spin_stats = on ? 1 : 0;
+  return VRAR_OK;
+}
+
+int vrar_get_spin_stats(uint64_t stats[5], int reset) {
+  if (!stats) return VRAR_EINVAL;
+  int dev = 0;
+  int rc = current_device(&dev);
+  if (rc != VRAR_OK) return rc;
+  std::memset(stats, 0, 5 * sizeof(uint64_t));
+  if (cudaDeviceSynchronize() != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& w = g_ws[dev];
+  if (!w.ctrl) return VRAR_OK;
+  unsigned long long h[kStCount];
+  if (cudaMemcpy(h, w.ctrl + kStats, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_fail(cudaErrorUnknown);
+  for (int i = 0; i < kStCount; ++i) stats[i] = h[i];
+  if (reset && cudaMemset(w.ctrl + kStats, 0, sizeof(h)) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
   return VRAR_OK;
 }
 
@@ -715,6 +760,6 @@ extern "C" int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* cons
   a.ctrl = reinterpret_cast<uint32_t*>(d->base);
   a.sig = nullptr;  // recursive doubling uses no barrier rows
   a.ll = reinterpret_cast<uint64_t*>(d->base + kNoAllocCtrlBytes);
-  a.B = blocks_per_rank((a.items + C - 1) / C, P, resident_ctas(fn, dev, d->sms));
+  a.B = blocks_per_rank((a.items + C - 1) / C, P, grid_budget(fn, dev, d->sms));
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
 }

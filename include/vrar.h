@@ -45,6 +45,9 @@
  *    and grown when a larger call needs more. Growing allocates, which is not
  *    allowed while a stream is being captured into a CUDA graph: make one call
  *    of the largest shape (or call vrar_reserve) before capturing.
+ *  - Settings (vrar_set_*) are read when a call is queued and become part of
+ *    that launch; a call captured into a CUDA graph keeps the settings it was
+ *    captured with.
  *  - Return value: VRAR_OK, or a negative VRAR_E* code. Argument errors are
  *    found on the host before anything is queued. A device wait that hits
  *    its time limit cannot be returned by the call that queued it: the kernel
@@ -168,6 +171,15 @@ VRAR_API int vrar_get_rd_chunks(void);
 VRAR_API int vrar_set_edge_sync(int on);
 VRAR_API int vrar_get_edge_sync(void);
 
+/* Upper bound on the CTAs one call launches (default 0 = as many as fit on
+ * the device at once; every call still gets at least one CTA per rank). A
+ * budget leaves SMs to work running concurrently on other streams, e.g. the
+ * partner micro-batch's GEMMs while this all-reduce runs on a communication
+ * stream; the all-reduce is bound by memory bandwidth, which a fraction of
+ * the SMs can already draw. Process-wide setting. */
+VRAR_API int vrar_set_max_ctas(int n);
+VRAR_API int vrar_get_max_ctas(void);
+
 /* Time limit of every device wait, in nanoseconds of %globaltimer
  * (default 2e9). Range 1e5 .. 6e10. */
 VRAR_API int vrar_set_spin_timeout_ns(uint64_t ns);
@@ -191,6 +203,22 @@ VRAR_API size_t vrar_workspace_bytes(int P, size_t n, vrar_dtype_t dtype, vrar_a
 /* Free the current device's workspace (synchronises the device). The next
  * call allocates a fresh, zeroed one. */
 VRAR_API int vrar_reset(void);
+
+/*
+ * Spin statistics of the cross-rank waits (flag barriers and payload polls),
+ * after the temporary instrumentation described in [CAR] "Validation": off by
+ * default; vrar_set_spin_stats(1) makes the following calls count, per wait,
+ * how many polls it took (one extra warp-level reduction and a few atomics per
+ * warp and wait). vrar_get_spin_stats waits for the device, then fills
+ *   stats[0] waits counted        stats[1] polls in total
+ *   stats[2] most polls in one wait
+ *   stats[3] waits of 16384 polls or more
+ *   stats[4] waits that hit the time limit (the "safety net")
+ * for the current device, and clears the counters if `reset` is non-zero.
+ * Returns VRAR_OK, VRAR_EINVAL (stats NULL) or VRAR_ECUDA.
+ */
+VRAR_API int vrar_set_spin_stats(int on);
+VRAR_API int vrar_get_spin_stats(uint64_t stats[5], int reset);
 
 /* Testing aid: ranks whose bit is set skip every flag post and payload send
  * of the following calls (until set back to 0), so that their peers' waits

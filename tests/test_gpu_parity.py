@@ -35,6 +35,7 @@ def _defaults():
         vrar.set_edge_sync(False)
         vrar.set_spin_timeout_ns(2_000_000_000)
         vrar.debug_set_fault_mask(0)
+        vrar.set_max_ctas(0)
 
 
 def _dev(xs_np, dtype):
@@ -305,6 +306,23 @@ def test_chunk_count_and_edge_sync_do_not_change_results():
         assert_bits(run(algo, xs, "bf16", edge=False), run(algo, xs, "bf16", edge=True), algo)
 
 
+@pytest.mark.parametrize("budget", [1, 16, 40])
+def test_cta_budget_keeps_results(budget):
+    """A CTA budget shrinks the grid (down to one CTA per rank); every
+    algorithm still matches the oracle."""
+    vrar.set_max_ctas(budget)
+    try:
+        for P, n in ((8, 300_007), (32, 70_001)):
+            xs = gen(P, n, "bf16", synth.normal(0.0, 1.0), seed=budget + P)
+            for algo, L in algos_for(P):
+                if algo == "hier" and L not in (1, P // 2):
+                    continue
+                assert_bits(run(algo, xs, "bf16", L=L), oracle.allreduce(algo, xs, "bf16", L=L),
+                            f"{algo} L={L} P={P} budget={budget}")
+    finally:
+        vrar.set_max_ctas(0)
+
+
 def test_shapes_interleaved_across_calls():
     """Flags and payload slots are reused across calls of different P, n and
     algorithm without ever being cleared."""
@@ -354,6 +372,50 @@ def test_device_argument_errors():
     assert e.value.code in (vrar.EINVAL, vrar.ENOTSUP)
 
 
+# ---- spin statistics ----------------------------------------------------------------------------
+
+def test_spin_stats_counts_every_wait():
+    vrar.get_spin_stats(reset=True)
+    P, n = 8, 8 * 4096  # 4096 items per rank: one item per thread, one chunk
+    xs = gen(P, n, "bf16", synth.normal(0.0, 1.0), seed=31)
+    run("rd", xs, "bf16")
+    assert vrar.get_spin_stats(reset=True)["waits"] == 0, "statistics must be off by default"
+    vrar.set_spin_stats(True)
+    try:
+        run("rd", xs, "bf16")
+        st = vrar.get_spin_stats(reset=True)
+        # every thread holding an item waits once per step: P * log2(P) * items
+        assert st["waits"] == P * 3 * 4096, st
+        assert st["polls"] >= st["waits"] and st["max_polls"] >= 1 and st["timeouts"] == 0, st
+        run("twostage", xs, "bf16")  # mid barrier: P polling threads per CTA
+        st = vrar.get_spin_stats(reset=True)
+        assert st["waits"] > 0 and st["waits"] % P == 0 and st["timeouts"] == 0, st
+        assert vrar.get_spin_stats()["waits"] == 0, "reset must clear the counters"
+    finally:
+        vrar.set_spin_stats(False)
+
+
+def test_spin_stats_count_timeouts():
+    xs = gen(4, 40_000, "bf16", synth.normal(0.0, 1.0), seed=32)
+    d_in = _dev(xs, "bf16")
+    vrar.get_spin_stats(reset=True)
+    vrar.set_spin_stats(True)
+    vrar.set_spin_timeout_ns(20_000_000)
+    vrar.debug_set_fault_mask(1 << 2)
+    try:
+        vrar.all_reduce(d_in, algo="rd")
+        rc, info = vrar.query_status()
+        assert rc == vrar.ETIMEDOUT
+        st = vrar.get_spin_stats(reset=True)
+        assert st["timeouts"] >= 1 and st["long_waits"] >= 1, st
+    finally:
+        vrar.set_spin_stats(False)
+        vrar.debug_set_fault_mask(0)
+    outs = vrar.all_reduce(d_in, algo="rd")
+    assert vrar.query_status()[0] == 0
+    assert_bits([to_np(o) for o in outs], oracle.allreduce("rd", xs, "bf16"), "rd after the timeout")
+
+
 # ---- failure detection: bounded waits, no GPU fault ----------------------------------------------
 
 @pytest.mark.parametrize("algo,P,L,edge,phase", [
@@ -381,3 +443,28 @@ def test_missing_rank_times_out_and_recovers(algo, P, L, edge, phase):
     rc, info = vrar.query_status()
     assert rc == 0, info
     assert_bits([to_np(o) for o in outs], oracle.allreduce(algo, xs, "bf16", L=L), f"{algo} after timeout")
+
+
+# ---- overlap with compute on another stream ------------------------------------------------------
+
+def test_allreduce_overlapped_with_gemm_on_another_stream():
+    """The all-reduce of one micro-batch runs on a side stream while the other
+    micro-batch's GEMMs run; every output must still equal the oracle's sum of
+    the partials (checked on sampled elements) on both micro-batches."""
+    import bench
+    m = bench.TboPrefill(torch.device("cuda", 0), P=8, tokens=1024, hidden=2048, layers=3)
+    comm = torch.cuda.Stream()
+    vrar.set_max_ctas(32)  # a budget leaves SMs to the GEMMs (and selects the deep pipeline)
+    try:
+        for _ in range(3):
+            m.step_overlapped(comm)
+        torch.cuda.synchronize()
+    finally:
+        vrar.set_max_ctas(0)
+    assert vrar.query_status()[0] == 0
+    rng = np.random.default_rng(5)
+    idx = torch.from_numpy(rng.integers(0, m.T * m.H, 50_000)).cuda()
+    for u in range(2):
+        parts = [to_np(p.reshape(-1)[idx]) for p in m.part[u]]
+        want = oracle.allreduce(vrar.select_algo(m.P, m.T * m.H), parts, "bf16")
+        assert_bits([to_np(o.reshape(-1)[idx]) for o in m.out[u]], want, f"micro-batch {u}")
