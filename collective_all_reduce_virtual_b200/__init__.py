@@ -29,7 +29,7 @@ OK, EINVAL, ENOTSUP, ENOMEM, ECUDA, ETIMEDOUT, ETOOBIG = 0, -1, -2, -3, -4, -5, 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 MAX_RANKS = 32
 
-DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1, torch.float16: 2}
 ALGOS = {"auto": 0, "oneshot": 1, "twostage": 2, "twostage_write": 3, "rd": 4, "hier": 5}
 ALGO_NAMES = {v: k for k, v in ALGOS.items()}
 
@@ -103,7 +103,7 @@ def _rank_tensors(ts: Sequence[torch.Tensor], numel: int | None, what: str):
         raise ValueError(f"{what}: need 1..{MAX_RANKS} rank tensors, got {len(ts)}")
     dt = ts[0].dtype
     if dt not in DTYPES:
-        raise TypeError(f"{what}: dtype must be bfloat16 or float32, got {dt}")
+        raise TypeError(f"{what}: dtype must be bfloat16, float16 or float32, got {dt}")
     dev = ts[0].device
     if dev.type != "cuda":
         raise ValueError(f"{what}: tensors must be on a CUDA device")

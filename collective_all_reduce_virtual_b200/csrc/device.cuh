@@ -21,6 +21,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace vrar {
@@ -225,6 +226,30 @@ struct Bf16T {
     __nv_bfloat16 h = __float2bfloat16_rn(f);
     return *reinterpret_cast<E*>(&h);
   }
+};
+
+// IEEE binary16: widening is exact (cvt.f32.f16), narrowing is round to
+// nearest even with subnormals kept (cvt.rn.f16x2.f32).
+struct F16T {
+  using E = uint16_t;
+  static constexpr int VE = 8;
+  __device__ __forceinline__ static void widen(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] & 0xFFFFu)));
+      f[2 * i + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] >> 16)));
+    }
+  }
+  __device__ __forceinline__ static uint32_t pack2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);  // .x (low half) = lo
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ __forceinline__ static uint4 narrow(const float (&f)[8]) {
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+  }
+  __device__ __forceinline__ static float elem_to_f(E e) { return __half2float(__ushort_as_half(e)); }
+  __device__ __forceinline__ static E f_to_elem(float f) { return __half_as_ushort(__float2half_rn(f)); }
 };
 
 struct F32T {

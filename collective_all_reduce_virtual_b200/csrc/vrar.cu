@@ -43,8 +43,9 @@ struct Workspace {
 std::mutex g_mu;
 Workspace g_ws[kMaxDevices];
 
-size_t elem_size(vrar_dtype_t dt) { return dt == VRAR_BF16 ? 2 : 4; }
-int64_t per_item(vrar_dtype_t dt) { return dt == VRAR_BF16 ? 8 : 4; }
+bool valid_dtype(vrar_dtype_t dt) { return dt == VRAR_BF16 || dt == VRAR_FP32 || dt == VRAR_FP16; }
+size_t elem_size(vrar_dtype_t dt) { return dt == VRAR_FP32 ? 4 : 2; }
+int64_t per_item(vrar_dtype_t dt) { return dt == VRAR_FP32 ? 4 : 8; }
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 int ilog2(int x) {
   int s = 0;
@@ -123,7 +124,7 @@ int check_buffers(const void* const in[], void* const out[], int P, size_t in_el
                   vrar_dtype_t dt) {
   if (!in || !out) return VRAR_EINVAL;
   if (P < 1 || P > kMaxRanks) return VRAR_EINVAL;
-  if (dt != VRAR_BF16 && dt != VRAR_FP32) return VRAR_EINVAL;
+  if (!valid_dtype(dt)) return VRAR_EINVAL;
   const size_t es = elem_size(dt);
   if (in_elems > (SIZE_MAX / 2) / es || out_elems > (SIZE_MAX / 2) / es) return VRAR_EINVAL;
   Range ri[kMaxRanks], ro[kMaxRanks];
@@ -359,11 +360,24 @@ constexpr int kWriteTileItems = 64;  // staged write mode: items per tile (1 KiB
 
 template <class D>
 KernelFn staged_kernel(int ti) {
-  switch (ti) {
-    case 32: return k_twostage_write_staged<D, 32>;
-    case 64: return k_twostage_write_staged<D, 64>;
-    default: return k_twostage_write_staged<D, 128>;
-  }
+  return ti == 64 ? k_twostage_write_staged<D, 64> : k_twostage_write_staged<D, 128>;
+}
+
+// Dispatch on the element type.
+KernelFn pick_kernel_dt(vrar_dtype_t dt, vrar_algo_t algo, int C) {
+  return dt == VRAR_BF16 ? pick_kernel<Bf16T>(algo, C) : dt == VRAR_FP16 ? pick_kernel<F16T>(algo, C)
+                                                                        : pick_kernel<F32T>(algo, C);
+}
+
+KernelFn staged_kernel_dt(vrar_dtype_t dt, int ti) {
+  return dt == VRAR_BF16 ? staged_kernel<Bf16T>(ti) : dt == VRAR_FP16 ? staged_kernel<F16T>(ti)
+                                                                      : staged_kernel<F32T>(ti);
+}
+
+int rd_chunks_for_dt(vrar_dtype_t dt, vrar_algo_t algo, int C, int64_t work, int P, int dev, int sms) {
+  return dt == VRAR_BF16   ? rd_chunks_for<Bf16T>(algo, C, work, P, dev, sms)
+         : dt == VRAR_FP16 ? rd_chunks_for<F16T>(algo, C, work, P, dev, sms)
+                           : rd_chunks_for<F32T>(algo, C, work, P, dev, sms);
 }
 
 const char* algo_name(int a) {
@@ -425,10 +439,9 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   if (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER) {
     const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
     const int64_t work = algo == VRAR_ALGO_RD ? items : (items + L - 1) / L;
-    C = dtype == VRAR_BF16 ? rd_chunks_for<Bf16T>(algo, C, work, P, dev, ws->sms)
-                           : rd_chunks_for<F32T>(algo, C, work, P, dev, ws->sms);
+    C = rd_chunks_for_dt(dtype, algo, C, work, P, dev, ws->sms);
   }
-  KernelFn fn = dtype == VRAR_BF16 ? pick_kernel<Bf16T>(algo, C) : pick_kernel<F32T>(algo, C);
+  KernelFn fn = pick_kernel_dt(dtype, algo, C);
   if (!fn) return VRAR_EINVAL;
 
   KArgs a;
@@ -475,7 +488,7 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     const int cap_budget = g_set.max_ctas.load();
     const bool deep = cap_budget > 0 && cap_budget <= ws->sms;
     const int ti = deep ? 128 : kWriteTileItems;
-    KernelFn sf = dtype == VRAR_BF16 ? staged_kernel<Bf16T>(ti) : staged_kernel<F32T>(ti);
+    KernelFn sf = staged_kernel_dt(dtype, ti);
     const int64_t tiles = std::max<int64_t>(1, (work + ti - 1) / ti);
     const int S = std::max(2, std::min(deep ? kMaxStages : 6, ((deep ? 192 : 96) * 1024) / (P * ti * 16)));
     const size_t smem = kStagedHeader + static_cast<size_t>(S) * P * ti * 16;
@@ -501,7 +514,9 @@ int vrar_reduce_scatter(const void* const rank_in[], void* const rank_out[], int
   if ((rc = current_device(&dev)) != VRAR_OK) return rc;
   Workspace* ws = nullptr;
   if ((rc = ensure_workspace(dev, 0, &ws)) != VRAR_OK) return rc;
-  KernelFn fn = dtype == VRAR_BF16 ? k_reduce_scatter<Bf16T> : k_reduce_scatter<F32T>;
+  KernelFn fn = dtype == VRAR_BF16   ? k_reduce_scatter<Bf16T>
+                : dtype == VRAR_FP16 ? k_reduce_scatter<F16T>
+                                     : k_reduce_scatter<F32T>;
   KArgs a;
   std::memset(&a, 0, sizeof(a));
   for (int p = 0; p < P; ++p) {
@@ -527,7 +542,9 @@ int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, 
   if ((rc = current_device(&dev)) != VRAR_OK) return rc;
   Workspace* ws = nullptr;
   if ((rc = ensure_workspace(dev, 0, &ws)) != VRAR_OK) return rc;
-  KernelFn fn = dtype == VRAR_BF16 ? k_all_gather<Bf16T> : k_all_gather<F32T>;
+  KernelFn fn = dtype == VRAR_BF16   ? k_all_gather<Bf16T>
+                : dtype == VRAR_FP16 ? k_all_gather<F16T>
+                                     : k_all_gather<F32T>;
   KArgs a;
   std::memset(&a, 0, sizeof(a));
   for (int p = 0; p < P; ++p) {
@@ -543,7 +560,7 @@ int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, 
 }
 
 int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype) {
-  if (P < 1 || P > kMaxRanks || (dtype != VRAR_BF16 && dtype != VRAR_FP32)) return VRAR_EINVAL;
+  if (P < 1 || P > kMaxRanks || !valid_dtype(dtype)) return VRAR_EINVAL;
   return select_algo(P, n, dtype);
 }
 
@@ -603,7 +620,7 @@ int vrar_reserve(size_t bytes) {
 }
 
 size_t vrar_workspace_bytes(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t algo) {
-  if (P < 1 || P > kMaxRanks || (dtype != VRAR_BF16 && dtype != VRAR_FP32)) return 0;
+  if (P < 1 || P > kMaxRanks || !valid_dtype(dtype)) return 0;
   if (algo == VRAR_ALGO_AUTO) algo = static_cast<vrar_algo_t>(select_algo(P, n, dtype));
   const int L = g_set.group_size.load();
   if (check_shape(algo, P, L) != VRAR_OK) return 0;
@@ -740,9 +757,8 @@ extern "C" int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* cons
   if ((rc = noalloc_setup(dev, &d)) != VRAR_OK) return rc;
 
   int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
-  C = dtype == VRAR_BF16 ? rd_chunks_for<Bf16T>(VRAR_ALGO_RD, C, items, P, dev, d->sms)
-                         : rd_chunks_for<F32T>(VRAR_ALGO_RD, C, items, P, dev, d->sms);
-  KernelFn fn = dtype == VRAR_BF16 ? pick_kernel<Bf16T>(VRAR_ALGO_RD, C) : pick_kernel<F32T>(VRAR_ALGO_RD, C);
+  C = rd_chunks_for_dt(dtype, VRAR_ALGO_RD, C, items, P, dev, d->sms);
+  KernelFn fn = pick_kernel_dt(dtype, VRAR_ALGO_RD, C);
   KArgs a;
   std::memset(&a, 0, sizeof(a));
   for (int p = 0; p < P; ++p) {

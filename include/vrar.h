@@ -31,9 +31,10 @@
  *    copied into the kernel's parameters by value, so they may be freed or
  *    reused as soon as the call returns.
  *  - n is the number of ELEMENTS of the full per-rank vector.
- *  - Elements are bf16 (VRAR_BF16) or IEEE binary32 (VRAR_FP32). Sums are
- *    formed in binary32 with round-to-nearest-even adds and rounded to the
- *    element type with round-to-nearest-even (subnormals kept).
+ *  - Elements are bf16 (VRAR_BF16), IEEE binary16 (VRAR_FP16) or IEEE
+ *    binary32 (VRAR_FP32). Sums are formed in binary32 with round-to-nearest-
+ *    even adds and rounded to the element type with round-to-nearest-even
+ *    (subnormals kept).
  *  - Out-of-place only: no output may overlap any input or another output.
  *  - 1 <= P <= VRAR_MAX_RANKS. n == 0 is a valid no-op.
  *  - The call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
@@ -78,7 +79,8 @@ typedef struct CUstream_st* vrar_stream_t;
 
 typedef enum {
     VRAR_BF16 = 0,
-    VRAR_FP32 = 1
+    VRAR_FP32 = 1,
+    VRAR_FP16 = 2   /* IEEE binary16 */
 } vrar_dtype_t;
 
 typedef enum {
@@ -240,7 +242,7 @@ VRAR_API int vrar_debug_set_fault_mask(uint32_t mask);
  * exits. It calls no cudaMalloc, no cudaFree and no allocating library routine.
  *  - Limit: P must be a power of two and
  *      256 + P * log2(P) * ceil(n / e) * 32 <= VRAR_NOALLOC_SCRATCH_BYTES,
- *    e = 8 for bf16, 4 for fp32 (for P = 8 and bf16: n <= 174,760). Larger
+ *    e = 8 for bf16 / fp16, 4 for fp32 (P = 8, bf16: n <= 174,760). Larger
  *    requests return VRAR_ETOOBIG before anything is queued.
  *  - The first call on a device sets that device up: it looks up the array's
  *    device address (cudaGetSymbolAddress) and zeroes it, which waits for the

@@ -4,8 +4,8 @@ TEST INFRASTRUCTURE ONLY: the tests, the package smoke check and the
 benchmark's CPU-baseline leg may use it; the product path never does. It is
 independent of the CUDA library (no shared code, headers or constants).
 
-Arrays are numpy: bf16 data travels as ``uint16`` bit patterns, fp32 as
-``float32``. A "rank list" is a list of P one-dimensional arrays.
+Arrays are numpy: bf16 and fp16 data travel as ``uint16`` bit patterns, fp32
+as ``float32``. A "rank list" is a list of P one-dimensional arrays.
 
 What each function computes, and which source passage it follows, is stated in
 oracle.cpp next to the C++ that does it. ``Oracle(path)`` wraps any build of
@@ -22,7 +22,7 @@ import numpy as np
 from . import build as _build
 
 ALGOS = ("oneshot", "twostage", "twostage_write", "rd", "hier")
-_NP = {"bf16": np.uint16, "fp32": np.float32}
+_NP = {"bf16": np.uint16, "fp16": np.uint16, "fp32": np.float32}
 
 
 def _ptrs(arrs):
@@ -51,6 +51,10 @@ class Oracle:
         L.oracle_bf16_round.restype = None
         L.oracle_bf16_widen.argtypes = [vp, vp, i64]
         L.oracle_bf16_widen.restype = None
+        L.oracle_fp16_round.argtypes = [vp, vp, i64]
+        L.oracle_fp16_round.restype = None
+        L.oracle_fp16_widen.argtypes = [vp, vp, i64]
+        L.oracle_fp16_widen.restype = None
         L.oracle_allreduce.argtypes = [cp, pp, pp, ctypes.c_int, i64, cp, ctypes.c_int, ctypes.c_int]
         L.oracle_allreduce.restype = ctypes.c_int
         L.oracle_reduce_scatter.argtypes = [pp, pp, ctypes.c_int, i64, cp]
@@ -74,6 +78,20 @@ class Oracle:
         h = np.ascontiguousarray(h, dtype=np.uint16)
         y = np.empty(h.shape, np.float32)
         self.lib.oracle_bf16_widen(h.ctypes.data, y.ctypes.data, h.size)
+        return y
+
+    def fp16_round(self, x: np.ndarray) -> np.ndarray:
+        """float32 -> fp16 bit patterns, round to nearest even (NaN -> 0x7E00)."""
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        y = np.empty(x.shape, np.uint16)
+        self.lib.oracle_fp16_round(x.ctypes.data, y.ctypes.data, x.size)
+        return y
+
+    def fp16_widen(self, h: np.ndarray) -> np.ndarray:
+        """fp16 bit patterns -> float32 (exact)."""
+        h = np.ascontiguousarray(h, dtype=np.uint16)
+        y = np.empty(h.shape, np.float32)
+        self.lib.oracle_fp16_widen(h.ctypes.data, y.ctypes.data, h.size)
         return y
 
     def allreduce(self, algo: str, xs, dtype: str = "bf16", L: int = 8, chunks: int = 4):
@@ -125,9 +143,11 @@ class Oracle:
         return S, A
 
     def to_float(self, x: np.ndarray, dtype: str) -> np.ndarray:
-        """Rank-buffer values as float64 (bf16 patterns widened exactly)."""
+        """Rank-buffer values as float64 (16-bit patterns widened exactly)."""
         if dtype == "bf16":
             return self.bf16_widen(x).astype(np.float64)
+        if dtype == "fp16":
+            return self.fp16_widen(x).astype(np.float64)
         return np.asarray(x, np.float64)
 
 
@@ -165,9 +185,17 @@ def bf16_widen(h):
     return default().bf16_widen(h)
 
 
+def fp16_round(x):
+    return default().fp16_round(x)
+
+
+def fp16_widen(h):
+    return default().fp16_widen(h)
+
+
 def to_float(x, dtype):
     return default().to_float(x, dtype)
 
 
 __all__ = ["ALGOS", "Oracle", "default", "allreduce", "reduce_scatter", "all_gather",
-           "fp64_reference", "bf16_round", "bf16_widen", "to_float"]
+           "fp64_reference", "bf16_round", "bf16_widen", "fp16_round", "fp16_widen", "to_float"]

@@ -24,8 +24,9 @@
  *           into every rank's registered output.
  *
  * Numerics (readings of the sources, which fix none of this):
- *  - Inputs are bf16 or fp32. Every add is one IEEE-754 binary32 add with
- *    round-to-nearest-even; a bf16 operand is widened exactly to fp32 first.
+ *  - Inputs are bf16, fp16 (IEEE binary16) or fp32. Every add is one IEEE-754
+ *    binary32 add with round-to-nearest-even; a 16-bit operand is widened
+ *    exactly to fp32 first.
  *  - A reduction of several ranks' values adds them left to right in
  *    ascending rank order starting from rank 0, and rounds once to the tensor
  *    type at the end.
@@ -33,10 +34,13 @@
  *    tensor-typed values in fp32 and rounds back to the tensor type.
  *  - fp32 -> bf16 is round-to-nearest-even from the definition of the format
  *    (bf16 = the upper 16 bits of a binary32); any NaN becomes 0x7FC0.
+ *  - fp32 -> fp16 is round-to-nearest-even from the definition of binary16
+ *    (1 sign, 5 exponent bits biased by 15, 10 fraction bits; subnormals in
+ *    steps of 2^-24; values from 65520 up round to infinity); NaN -> 0x7E00.
  *
  * Floating-point environment: the functions below clear the x86 flush-to-zero
- * and denormals-are-zero bits for their duration, so subnormal bf16/fp32
- * inputs are added exactly as IEEE-754 says, whatever the caller left set.
+ * and denormals-are-zero bits for their duration, so subnormal inputs and
+ * sums are handled exactly as IEEE-754 says, whatever the caller left set.
  */
 
 #include <cstddef>
@@ -91,12 +95,55 @@ inline uint16_t bf16_round(float f) {
     return static_cast<uint16_t>(u >> 16);
 }
 
+/* binary16 -> binary32, exact. Subnormal halves are fraction * 2^-24 (a
+ * product of an integer below 1024 and a power of two: exact in binary32). */
+inline float half_widen(uint16_t h) {
+    const uint32_t sign = static_cast<uint32_t>(h & 0x8000u) << 16;
+    const uint32_t exp = (h >> 10) & 0x1Fu, frac = h & 0x3FFu;
+    if (exp == 0) {
+        const float v = static_cast<float>(frac) * (1.0f / 16777216.0f);
+        return sign ? -v : v;
+    }
+    if (exp == 31) return bits_to_f32(sign | 0x7F800000u | (frac << 13));
+    return bits_to_f32(sign | ((exp + 112u) << 23) | (frac << 13));
+}
+
+/* binary32 -> binary16, round to nearest, ties to even. */
+inline uint16_t half_round(float f) {
+    const uint32_t u = f32_to_bits(f);
+    const uint16_t sign = static_cast<uint16_t>((u >> 16) & 0x8000u);
+    const uint32_t a = u & 0x7FFFFFFFu;
+    if (a > 0x7F800000u) return 0x7E00u;                        // NaN
+    if (a >= 0x477FF000u) return static_cast<uint16_t>(sign | 0x7C00u);  // >= 65520 (and inf) -> inf
+    if (a >= 0x38800000u) {                                     // >= 2^-14: a normal half
+        const uint32_t m = a - 0x38000000u;                     // exponent rebias 127 -> 15
+        uint32_t keep = m >> 13;
+        const uint32_t rest = m & 0x1FFFu;
+        if (rest > 0x1000u || (rest == 0x1000u && (keep & 1u))) keep += 1;  // a carry may step the exponent
+        return static_cast<uint16_t>(sign | keep);
+    }
+    // Subnormal (or zero) half: round |f| / 2^-24 to an integer, ties to even.
+    // The scaling by a power of two is exact, and so is the fraction below.
+    const float q = bits_to_f32(a) * 16777216.0f;
+    uint32_t i = static_cast<uint32_t>(q);
+    const float rest = q - static_cast<float>(i);
+    if (rest > 0.5f || (rest == 0.5f && (i & 1u))) i += 1;     // i may reach 1024 = the smallest normal
+    return static_cast<uint16_t>(sign | i);
+}
+
 /* ---- element types ------------------------------------------------------------ */
 
 struct Bf16 {
     using T = uint16_t;
     static float widen(T v) { return bf16_widen(v); }
     static T narrow(float a) { return bf16_round(a); }
+    static constexpr int64_t bytes = 2;
+};
+
+struct F16 {
+    using T = uint16_t;
+    static float widen(T v) { return half_widen(v); }
+    static T narrow(float a) { return half_round(a); }
     static constexpr int64_t bytes = 2;
 };
 
@@ -272,11 +319,21 @@ void all_gather(const void* const* in, void* const* out, int P, int64_t n) {
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
+enum Dt { DT_BF16 = 0, DT_F16 = 1, DT_F32 = 2 };
+
 int dtype_code(const char* dt) {
     if (!dt) return -1;
-    if (std::strcmp(dt, "bf16") == 0) return 2;
-    if (std::strcmp(dt, "fp32") == 0) return 4;
+    if (std::strcmp(dt, "bf16") == 0) return DT_BF16;
+    if (std::strcmp(dt, "fp16") == 0) return DT_F16;
+    if (std::strcmp(dt, "fp32") == 0) return DT_F32;
     return -1;
+}
+
+/* Element value of buffer x at index i as double (exact for all three types). */
+double elem_as_double(const void* x, int64_t i, int dt) {
+    if (dt == DT_BF16) return static_cast<double>(bf16_widen(static_cast<const uint16_t*>(x)[i]));
+    if (dt == DT_F16) return static_cast<double>(half_widen(static_cast<const uint16_t*>(x)[i]));
+    return static_cast<double>(static_cast<const float*>(x)[i]);
 }
 
 template <class E>
@@ -312,10 +369,22 @@ void oracle_bf16_widen(const uint16_t* x, float* y, int64_t n) {
     for (int64_t i = 0; i < n; ++i) y[i] = bf16_widen(x[i]);
 }
 
+/* Round n binary32 values to fp16 bit patterns. */
+void oracle_fp16_round(const float* x, uint16_t* y, int64_t n) {
+    IeeeScope env;
+    for (int64_t i = 0; i < n; ++i) y[i] = half_round(x[i]);
+}
+
+/* Widen n fp16 bit patterns to binary32. */
+void oracle_fp16_widen(const uint16_t* x, float* y, int64_t n) {
+    IeeeScope env;
+    for (int64_t i = 0; i < n; ++i) y[i] = half_widen(x[i]);
+}
+
 /* All-reduce of P rank buffers of n elements. algo: "oneshot", "twostage",
- * "twostage_write", "rd", "hier"; dtype: "bf16" (uint16 bit patterns) or
- * "fp32". L is the group size for "hier"; chunks is the chunk count of the
- * recursive-doubling phase. Returns 0, -1 (bad argument) or -2 (P/L shape the
+ * "twostage_write", "rd", "hier"; dtype: "bf16" or "fp16" (uint16 bit
+ * patterns) or "fp32". L is the group size for "hier"; chunks is the chunk
+ * count of the recursive-doubling phase. Returns 0, -1 (bad argument) or -2 (P/L shape the
  * algorithm does not define). */
 int oracle_allreduce(const char* algo, const void* const* in, void* const* out, int P, int64_t n,
                      const char* dtype, int L, int chunks) {
@@ -323,8 +392,9 @@ int oracle_allreduce(const char* algo, const void* const* in, void* const* out, 
     const int dt = dtype_code(dtype);
     if (!algo || !in || !out || P < 1 || n < 0 || dt < 0) return -1;
     if (n == 0) return 0;
-    return dt == 2 ? allreduce_t<Bf16>(algo, in, out, P, n, L, chunks)
-                   : allreduce_t<F32>(algo, in, out, P, n, L, chunks);
+    if (dt == DT_BF16) return allreduce_t<Bf16>(algo, in, out, P, n, L, chunks);
+    if (dt == DT_F16) return allreduce_t<F16>(algo, in, out, P, n, L, chunks);
+    return allreduce_t<F32>(algo, in, out, P, n, L, chunks);
 }
 
 /* Reduce-scatter: in[p] has n elements, out[p] has n / P; n % P == 0. */
@@ -332,7 +402,9 @@ int oracle_reduce_scatter(const void* const* in, void* const* out, int P, int64_
     IeeeScope env;
     const int dt = dtype_code(dtype);
     if (!in || !out || P < 1 || n < 0 || dt < 0 || n % P != 0) return -1;
-    if (dt == 2) reduce_scatter<Bf16>(in, out, P, n); else reduce_scatter<F32>(in, out, P, n);
+    if (dt == DT_BF16) reduce_scatter<Bf16>(in, out, P, n);
+    else if (dt == DT_F16) reduce_scatter<F16>(in, out, P, n);
+    else reduce_scatter<F32>(in, out, P, n);
     return 0;
 }
 
@@ -340,7 +412,9 @@ int oracle_reduce_scatter(const void* const* in, void* const* out, int P, int64_
 int oracle_all_gather(const void* const* in, void* const* out, int P, int64_t n, const char* dtype) {
     const int dt = dtype_code(dtype);
     if (!in || !out || P < 1 || n < 0 || dt < 0 || n % P != 0) return -1;
-    if (dt == 2) all_gather<Bf16>(in, out, P, n); else all_gather<F32>(in, out, P, n);
+    if (dt == DT_BF16) all_gather<Bf16>(in, out, P, n);
+    else if (dt == DT_F16) all_gather<F16>(in, out, P, n);
+    else all_gather<F32>(in, out, P, n);
     return 0;
 }
 
@@ -354,8 +428,7 @@ int oracle_fp64_reference(const void* const* in, int P, int64_t n, const char* d
     for (int64_t i = 0; i < n; ++i) {
         double s = 0.0, a = 0.0;
         for (int p = 0; p < P; ++p) {
-            double x = dt == 2 ? static_cast<double>(bf16_widen(static_cast<const uint16_t*>(in[p])[i]))
-                               : static_cast<double>(static_cast<const float*>(in[p])[i]);
+            const double x = elem_as_double(in[p], i, dt);
             s += x;
             a += x < 0 ? -x : x;
         }

@@ -24,8 +24,8 @@ Distributions (element i of rank r):
   ``z = sqrt(-2 ln U1) * cos(2 pi U2)``, value ``mu + sigma * z``.
 
 The float64 value is then rounded to float32 (round to nearest even) and, for
-bf16 tensors, from float32 to bf16 (round to nearest even). Integer values in
--8..8 are exact in both types.
+bf16 or fp16 tensors, from float32 to that type (round to nearest even).
+Integer values in -8..8 are exact in all three types.
 
 Everything is written with int64 torch ops (two's-complement wrap-around
 stands in for unsigned 64-bit arithmetic), so it runs unchanged on the CPU or
@@ -157,12 +157,12 @@ def rank_values(dist: Dist, seed: int, rank: int, idx: torch.Tensor) -> torch.Te
 
 
 def to_dtype(v64: torch.Tensor, dtype: torch.dtype) -> torch.Tensor:
-    """float64 -> float32 (RNE) -> dtype (RNE); bf16 and fp32 only."""
+    """float64 -> float32 (RNE) -> dtype (RNE); bf16, fp16 and fp32."""
     v32 = v64.to(torch.float32)
     if dtype == torch.float32:
         return v32
-    if dtype == torch.bfloat16:
-        return v32.to(torch.bfloat16)
+    if dtype in (torch.bfloat16, torch.float16):
+        return v32.to(dtype)
     raise ValueError(f"unsupported dtype {dtype}")
 
 

@@ -4,7 +4,8 @@ Each ``pin_*`` takes an ``oracle.Oracle`` and raises AssertionError when the
 oracle disagrees with what the mathematics or the sources fix:
 
 * torch's float32 -> bfloat16 conversion (a library routine for the textbook
-  round-to-nearest-even) on every bf16 boundary pattern;
+  round-to-nearest-even) on every bf16 boundary pattern, and numpy's
+  float32 -> float16 conversion on every tie point of every binary16 value;
 * exact integer sums (every algorithm must return the exact sum of small
   integers, which bf16 and fp32 hold exactly) by brute force;
 * closed forms of a periodic integer pattern;
@@ -96,8 +97,50 @@ def pin_bf16_widen(o):
     assert (ours == (h.astype(np.uint32) << 16)).all(), "widening appends 16 zero bits"
 
 
+def pin_fp16_round_vs_numpy(o):
+    """Every tie point and its neighbours for every finite binary16 value (both
+    signs), plus random binary32 patterns, against numpy's float32 -> float16
+    conversion (a library routine for round-to-nearest-even)."""
+    h = np.arange(0x7C00, dtype=np.uint32).astype(np.uint16)            # finite, positive
+    lo = h.view(np.float16).astype(np.float32)
+    hi = (h.astype(np.uint32) + 1).astype(np.uint16).view(np.float16).astype(np.float32)
+    mid = (lo.astype(np.float64) + hi.astype(np.float64)) / 2            # exact in binary32
+    mid32 = mid.astype(np.float32)
+    assert (mid32.astype(np.float64) == mid).all()
+    pts = [lo, mid32, np.nextafter(mid32, np.float32(0)), np.nextafter(mid32, np.float32(np.inf))]
+    x = np.concatenate(pts)
+    x = np.concatenate([x, -x])
+    rng = np.random.default_rng(7)
+    x = np.concatenate([x, rng.integers(0, 2**32, 500_000, dtype=np.uint64).astype(np.uint32).view(np.float32)])
+    with np.errstate(over="ignore", invalid="ignore"):
+        ref = x.astype(np.float16).view(np.uint16)
+    ours = o.fp16_round(x)
+    nan = np.isnan(x)
+    assert (ours[~nan] == ref[~nan]).all(), "fp16 rounding differs from numpy"
+    assert (ours[nan] == 0x7E00).all()
+
+
+def pin_fp16_widen(o):
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = o.fp16_widen(h)
+    ref = h.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert (ours.view(np.uint32)[~nan] == ref.view(np.uint32)[~nan]).all()
+
+
+def pin_fp16_round_hand(o):
+    cases = [(1.0, 0x3C00), (1.0 + 2**-11, 0x3C00), (1.0 + 3 * 2**-11, 0x3C02), (65504.0, 0x7BFF),
+             (65519.0, 0x7BFF), (65520.0, 0x7C00), (2**-24, 0x0001), (2**-25, 0x0000), (3 * 2**-26, 0x0001),
+             (1.5 * 2**-24, 0x0002), (2**-14, 0x0400), (2**-14 - 2**-25, 0x0400), (-0.0, 0x8000),
+             (-(1.0 + 2**-11), 0xBC00)]
+    x = np.array([c[0] for c in cases], np.float32)
+    want = np.array([c[1] for c in cases], np.uint16)
+    assert (o.fp16_round(x) == want).all()
+
+
 def pin_integer_sums(o, n_values=tuple(range(1, 68)), P_values=(1, 2, 3, 4, 5, 8, 16, 32)):
-    for dtype in ("bf16", "fp32"):
+    for dtype in ("bf16", "fp32", "fp16"):
         for P in P_values:
             for n in n_values:
                 xs = gen(P, n, dtype, synth.INT8, seed=1000 + P * 97 + n)
@@ -126,10 +169,11 @@ def pin_closed_form(o):
         16: 8 - ((10 + i) % 17),
         32: 16 - ((3 + i) % 17) - ((10 + i) % 17),
     }
-    for dtype in ("bf16", "fp32"):
+    for dtype in ("bf16", "fp32", "fp16"):
         for P, want in closed.items():
             vals = [(((7 * p + i) % 17) - 8).astype(np.float32) for p in range(P)]
-            xs = [(v.view(np.uint32) >> 16).astype(np.uint16) if dtype == "bf16" else v for v in vals]
+            xs = [(v.view(np.uint32) >> 16).astype(np.uint16) if dtype == "bf16"
+                  else v.astype(np.float16).view(np.uint16) if dtype == "fp16" else v for v in vals]
             for algo, L in _algos_for(P):
                 outs = o.allreduce(algo, xs, dtype, L=L)
                 got = o.to_float(outs[0], dtype)
@@ -154,8 +198,8 @@ def pin_golden_order(o):
 def pin_error_bound(o):
     """|y - S| <= rtol * A with S, A from math.fsum (independent of the oracle's
     own fp64 helper, which is checked here too)."""
-    rtol = {"bf16": 1e-2, "fp32": 1e-5}
-    for dtype in ("bf16", "fp32"):
+    rtol = {"bf16": 1e-2, "fp32": 1e-5, "fp16": 5e-3}
+    for dtype in ("bf16", "fp32", "fp16"):
         for P in (2, 8, 32):
             n = 300
             xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=7 + P)
@@ -183,7 +227,7 @@ def pin_fp32_left_fold(o):
 
 
 def pin_invariants(o):
-    for dtype in ("bf16", "fp32"):
+    for dtype in ("bf16", "fp32", "fp16"):
         for P in (1, 2, 4, 8, 32):
             n = 531  # several 16-byte vectors, a ragged tail
             xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=40 + P)
@@ -207,7 +251,7 @@ def pin_invariants(o):
 
 
 def pin_rs_ag(o):
-    for dtype in ("bf16", "fp32"):
+    for dtype in ("bf16", "fp32", "fp16"):
         for P in (1, 2, 3, 8, 32):
             m = 37
             n = m * P
@@ -250,6 +294,9 @@ ALL_PINS = [
     pin_bf16_round_vs_torch,
     pin_bf16_round_hand,
     pin_bf16_widen,
+    pin_fp16_round_vs_numpy,
+    pin_fp16_widen,
+    pin_fp16_round_hand,
     pin_integer_sums,
     pin_closed_form,
     pin_golden_order,

@@ -136,7 +136,7 @@ def test_settings_round_trip_and_ranges():
 def test_selector_is_defined_for_every_shape():
     for P in range(1, 33):
         for n in (1, 1000, 65536, 1 << 20, 117440512):
-            for dt in (torch.bfloat16, torch.float32):
+            for dt in (torch.bfloat16, torch.float32, torch.float16):
                 a = vrar.select_algo(P, n, dt)
                 assert a in ("oneshot", "twostage", "twostage_write", "rd", "hier")
                 if a == "rd":
@@ -154,6 +154,7 @@ def test_selector_table_entries():
     assert vrar.select_algo(8, 117440512, bf) == "twostage_write"   # prefill
     assert vrar.select_algo(32, 16384, bf) == "twostage_write"      # 32 KiB at 32 ranks
     assert vrar.select_algo(8, 65536, torch.float32) == "oneshot"   # 256 KiB in fp32
+    assert vrar.select_algo(8, 524288, torch.float16) == "twostage_write"
 
 
 def test_workspace_bytes():

@@ -23,7 +23,7 @@ if torch.cuda.is_available():
 else:  # collected on the CPU machine, never run there
     vrar = None
 
-RTOL = {"bf16": 1e-2, "fp32": 1e-5}
+RTOL = {"bf16": 1e-2, "fp32": 1e-5, "fp16": 5e-3}
 
 
 @pytest.fixture(autouse=True)
@@ -74,7 +74,7 @@ SHAPES = [(P, n) for P in (1, 2, 3, 4, 5, 8) for n in (1, 7, 8, 9, 4099, 100_003
          [(P, n) for P in (16, 32) for n in (1, 9, 20_011)]
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32", "fp16"])
 @pytest.mark.parametrize("P,n", SHAPES)
 def test_parity_small(P, n, dtype):
     xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P * 1000 + n)
@@ -84,7 +84,7 @@ def test_parity_small(P, n, dtype):
         assert_bits(got, want, f"{algo} L={L} P={P} n={n} {dtype}")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32", "fp16"])
 def test_integer_inputs_give_exact_sums(dtype):
     for P in (2, 4, 8, 16, 32):
         n = 5003
@@ -107,7 +107,7 @@ def test_golden_order_cases_on_gpu():
             assert_bits(got, [want] * len(got), f"{case['name']} {spec}")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32", "fp16"])
 def test_fp64_tolerance(dtype):
     for P in (2, 8, 32):
         xs = gen(P, 30_000, dtype, synth.normal(0.0, 1.0), seed=77 + P)
@@ -122,8 +122,9 @@ def test_special_values_classes():
     vals = np.array([np.inf, -np.inf, 1e-40, -1e-40, 0.0, -0.0, 3e38, 3e38], np.float32)
     xs32 = [vals, np.array([1.0, 1.0, 1e-40, 0.0, -0.0, -0.0, 3e38, -3e38], np.float32),
             np.array([-np.inf, 2.0, 0.0, -1e-40, -0.0, -0.0, 0.0, 1.0], np.float32)]
-    for dtype in ("fp32", "bf16"):
-        xs = xs32 if dtype == "fp32" else [oracle.bf16_round(x) for x in xs32]
+    for dtype in ("fp32", "bf16", "fp16"):
+        xs = xs32 if dtype == "fp32" else [oracle.bf16_round(x) if dtype == "bf16" else oracle.fp16_round(x)
+                                           for x in xs32]
         for algo in ("oneshot", "twostage", "twostage_write"):
             want = oracle.allreduce(algo, xs, dtype)
             got = run(algo, xs, dtype)
@@ -334,7 +335,7 @@ def test_shapes_interleaved_across_calls():
         assert_bits(run(algo, xs, "bf16", L=L), oracle.allreduce(algo, xs, "bf16", L=L), f"step {i} {algo}")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32", "fp16"])
 def test_reduce_scatter_and_all_gather(dtype):
     for P in (1, 2, 3, 8, 32):
         for m in (8, 37, 4104, 20_000):

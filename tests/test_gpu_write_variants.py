@@ -25,7 +25,7 @@ CHILD = textwrap.dedent("""
     import collective_all_reduce_virtual_b200 as vrar
     import oracle, synth
     from util import from_np, gen, to_np, bits_of
-    for dtype in ("bf16", "fp32"):
+    for dtype in ("bf16", "fp32", "fp16"):
         for P, n in ((1, 1001), (2, 7), (3, 66_001), (8, 9), (8, 300_007), (16, 70_001), (32, 33_333), (32, 1_000_003)):
             xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P + n)
             want = oracle.allreduce("twostage_write", xs, dtype)

@@ -41,6 +41,12 @@ MUTANTS = {
                               "out_ptr<E>(out, p)[j * P + c] = in_ptr<E>(in, c)[j];"),
     "reduce_scatter_strided": ("reduce_ranks<E>(in, 0, P, p * m + j);", "reduce_ranks<E>(in, 0, P, j * P + p);"),
     "fp64_scale_signed": ("a += x < 0 ? -x : x;", "a += x;"),
+    "half_round_half_away": ("if (rest > 0x1000u || (rest == 0x1000u && (keep & 1u))) keep += 1;",
+                             "if (rest >= 0x1000u) keep += 1;"),
+    "half_subnormal_truncate": ("if (rest > 0.5f || (rest == 0.5f && (i & 1u))) i += 1;",
+                                "if (rest > 2.0f) i += 1;"),
+    "half_widen_bias": ("return bits_to_f32(sign | ((exp + 112u) << 23) | (frac << 13));",
+                        "return bits_to_f32(sign | ((exp + 111u) << 23) | (frac << 13));"),
 }
 
 

@@ -11,22 +11,22 @@ import torch
 import synth
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
-TORCH_DT = {"bf16": torch.bfloat16, "fp32": torch.float32}
-NP_DT = {"bf16": np.uint16, "fp32": np.float32}
+TORCH_DT = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
+NP_DT = {"bf16": np.uint16, "fp16": np.uint16, "fp32": np.float32}
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
-    """A CPU tensor's elements as numpy: bf16 as uint16 bit patterns."""
+    """A CPU tensor's elements as numpy: bf16 / fp16 as uint16 bit patterns."""
     t = t.detach().cpu().contiguous()
-    if t.dtype == torch.bfloat16:
+    if t.dtype in (torch.bfloat16, torch.float16):
         return t.view(torch.int16).numpy().view(np.uint16).copy()
     return t.numpy().copy()
 
 
 def from_np(a: np.ndarray, dtype: str) -> torch.Tensor:
-    """numpy rank buffer (uint16 patterns for bf16) -> CPU tensor of that dtype."""
-    if dtype == "bf16":
-        return torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16).copy()).view(torch.bfloat16)
+    """numpy rank buffer (uint16 patterns for 16-bit types) -> CPU tensor of that dtype."""
+    if dtype in ("bf16", "fp16"):
+        return torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16).copy()).view(TORCH_DT[dtype])
     return torch.from_numpy(np.ascontiguousarray(a, np.float32).copy())
 
 
@@ -42,6 +42,10 @@ def hexvals(strs, dtype: str) -> np.ndarray:
     assert (f32.astype(np.float64) == f).all(), "fixture value not exact in fp32"
     if dtype == "fp32":
         return f32
+    if dtype == "fp16":
+        h = f32.astype(np.float16)
+        assert (h.astype(np.float64) == f).all(), "fixture value not exact in fp16"
+        return h.view(np.uint16)
     bits = f32.view(np.uint32)
     assert (bits & 0xFFFF == 0).all(), "fixture value not exact in bf16"
     return (bits >> 16).astype(np.uint16)
