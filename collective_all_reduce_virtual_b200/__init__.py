@@ -45,6 +45,8 @@ SIGNATURES = {
     "vrar_get_group_size": ([], _i),
     "vrar_set_rd_chunks": ([_i], _i),
     "vrar_get_rd_chunks": ([], _i),
+    "vrar_set_payload_wire": ([_i], _i),
+    "vrar_get_payload_wire": ([], _i),
     "vrar_set_edge_sync": ([_i], _i),
     "vrar_get_edge_sync": ([], _i),
     "vrar_set_max_ctas": ([_i], _i),
@@ -190,6 +192,18 @@ def get_rd_chunks() -> int:
     return _lib.vrar_get_rd_chunks()
 
 
+WIRE_ELEMENT, WIRE_FP32 = 0, 1
+
+
+def set_payload_wire(wire: str) -> None:
+    """'element' (default) or 'fp32': what RD / HIER payload words carry."""
+    _check(_lib.vrar_set_payload_wire({"element": WIRE_ELEMENT, "fp32": WIRE_FP32}[wire]), "vrar_set_payload_wire")
+
+
+def get_payload_wire() -> str:
+    return "fp32" if _lib.vrar_get_payload_wire() == WIRE_FP32 else "element"
+
+
 def set_edge_sync(on: bool) -> None:
     _check(_lib.vrar_set_edge_sync(1 if on else 0), "vrar_set_edge_sync")
 
@@ -261,7 +275,7 @@ def version() -> int:
 
 
 __all__ = ["all_reduce", "reduce_scatter", "all_gather", "select_algo", "set_group_size",
-           "get_group_size", "set_rd_chunks", "get_rd_chunks", "set_edge_sync", "get_edge_sync",
+           "get_group_size", "set_rd_chunks", "get_rd_chunks", "set_payload_wire", "get_payload_wire", "set_edge_sync", "get_edge_sync",
            "set_max_ctas", "get_max_ctas", "set_spin_timeout_ns", "get_spin_timeout_ns", "query_status", "reserve",
            "workspace_bytes", "reset", "set_spin_stats", "get_spin_stats", "debug_set_fault_mask", "strerror", "version", "VrarError",
            "ALGOS", "DTYPES", "SIGNATURES", "LIB_PATH", "lib", "ptr_array"]

@@ -337,11 +337,11 @@ __device__ __forceinline__ void store_item(void* base, int64_t it, int64_t n, co
   for (int i = 0; i < nv; ++i) p[i] = t.e[i];
 }
 
-// Ascending-rank fp32 sum of item `it` over ranks first .. first+count-1, one
-// rounding. Loads are issued eight at a time so that they overlap; the adds
+// Ascending-rank fp32 sum of item `it` over ranks first .. first+count-1 (not
+// rounded). Loads are issued eight at a time so that they overlap; the adds
 // stay in rank order.
 template <class D>
-__device__ __forceinline__ uint4 reduce_item(const RankPtrs& rp, int first, int count, int64_t it, int64_t n) {
+__device__ __forceinline__ Acc<D> reduce_item_acc(const RankPtrs& rp, int first, int count, int64_t it, int64_t n) {
   Acc<D> acc;
   for (int q0 = 0; q0 < count; q0 += 8) {
     uint4 x[8];
@@ -355,7 +355,26 @@ __device__ __forceinline__ uint4 reduce_item(const RankPtrs& rp, int first, int 
       }
     }
   }
-  return acc.round();
+  return acc;
+}
+
+// The same sum rounded once to the element type.
+template <class D>
+__device__ __forceinline__ uint4 reduce_item(const RankPtrs& rp, int first, int count, int64_t it, int64_t n) {
+  return reduce_item_acc<D>(rp, first, count, it, n).round();
+}
+
+// A 16-byte item of a 16-bit type as fp32 partials: two quads of 4 floats.
+__device__ __forceinline__ void floats_to_quads(const float (&f)[8], uint4& q0, uint4& q1) {
+  q0 = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+  q1 = make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]), __float_as_uint(f[7]));
+}
+
+template <class D>
+__device__ __forceinline__ uint4 quads_to_item(const uint4& q0, const uint4& q1) {
+  const float f[8] = {__uint_as_float(q0.x), __uint_as_float(q0.y), __uint_as_float(q0.z), __uint_as_float(q0.w),
+                      __uint_as_float(q1.x), __uint_as_float(q1.y), __uint_as_float(q1.z), __uint_as_float(q1.w)};
+  return D::narrow(f);
 }
 
 // ---- launch ordering -------------------------------------------------------------------

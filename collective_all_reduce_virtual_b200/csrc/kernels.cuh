@@ -451,6 +451,109 @@ __global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
   }
 }
 
+// Recursive doubling and the hierarchical all-reduce with fp32 partials on
+// the wire (16-bit element types). Each 16-byte input item becomes two fp32
+// quads that travel as fused payload words exactly like fp32 elements (so
+// twice the payload words of the element-type wire); the steps add in fp32
+// without rounding, and the store rounds once to the element type. Slots hold
+// 2 quads per item. C is at most 2 here (2C quads in flight per thread).
+template <class D, int C>
+__global__ void __launch_bounds__(kThreads) k_rd_wide(const KArgs a) {
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
+  const int64_t per_chunk = (a.items + C - 1) / C;
+  if (threadIdx.x < C) {
+    const int64_t first = threadIdx.x * per_chunk + static_cast<int64_t>(c.b) * kThreads;
+    const int64_t count = min(static_cast<int64_t>(kThreads), (threadIdx.x + 1) * per_chunk - first);
+    prefetch_items<D>(a.ptr.in[c.r], first, count, a.n);
+  }
+  pdl_wait();
+  const unsigned long long ticket = cta_take_ticket(a);
+  bool ok = true;
+  for (int64_t base = 0; base < per_chunk; base += stride) {  // same trip count in the whole CTA
+    const int64_t j = base + t0;
+    uint4 q[2 * C];
+    int64_t qidx[2 * C];
+    bool qval[2 * C];
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      const int64_t idx = k * per_chunk + j;
+      const bool val = ok && j < per_chunk && idx < a.items;
+      qidx[2 * k] = 2 * idx;
+      qidx[2 * k + 1] = 2 * idx + 1;
+      qval[2 * k] = qval[2 * k + 1] = val;
+      if (val) {
+        Acc<D> x;
+        x.init(load_item_input<D>(a.ptr.in[c.r], idx, a.n));
+        floats_to_quads(x.v, q[2 * k], q[2 * k + 1]);
+      }
+    }
+    if (base == 0) cta_publish_flag(c, ticket);
+    if (!ok) continue;
+    ok = rd_exchange<F32T, 2 * C, false>(a, c, q, qidx, qval, 2 * a.items);
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < C; ++k)
+        if (qval[2 * k]) store_item<D, true>(a.ptr.out[c.r], qidx[2 * k] / 2, a.n, quads_to_item<D>(q[2 * k], q[2 * k + 1]));
+    }
+  }
+}
+
+template <class D, int C>
+__global__ void __launch_bounds__(kThreads) k_hier_wide(const KArgs a) {
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const int L = a.L, g = c.r / L, l = c.r % L;
+  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
+  const int64_t piece = (a.items + L - 1) / L;
+  const int64_t lo = lo_of(l, piece, a.items), len = lo_of(l + 1, piece, a.items) - lo;
+  const int64_t per_chunk = (len + C - 1) / C;
+  if (threadIdx.x < L * C) {
+    const int k = threadIdx.x % C;
+    const int64_t first = k * per_chunk + static_cast<int64_t>(c.b) * kThreads;
+    const int64_t count = min(static_cast<int64_t>(kThreads), min((k + 1) * per_chunk, len) - first);
+    prefetch_items<D>(a.ptr.in[g * L + threadIdx.x / C], lo + first, count, a.n);
+  }
+  pdl_wait();
+  const unsigned long long ticket = cta_take_ticket(a);
+  bool ok = true;
+  for (int64_t base = 0; base < per_chunk; base += stride) {  // same trip count in the whole CTA
+    const int64_t j = base + t0;
+    uint4 q[2 * C];
+    int64_t qidx[2 * C];
+    bool qval[2 * C];
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      const int64_t idx = k * per_chunk + j;
+      const bool val = ok && j < per_chunk && idx < len;
+      qidx[2 * k] = 2 * idx;
+      qidx[2 * k + 1] = 2 * idx + 1;
+      qval[2 * k] = qval[2 * k + 1] = val;
+      if (val) {
+        const Acc<D> s = reduce_item_acc<D>(a.ptr, g * L, L, lo + idx, a.n);  // not rounded
+        floats_to_quads(s.v, q[2 * k], q[2 * k + 1]);
+      }
+    }
+    if (base == 0) cta_publish_flag(c, ticket);
+    if (!ok) continue;
+    ok = rd_exchange<F32T, 2 * C, true>(a, c, q, qidx, qval, 2 * piece);
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < C; ++k) {
+        if (!qval[2 * k]) continue;
+        const uint4 v = quads_to_item<D>(q[2 * k], q[2 * k + 1]);
+        for (int jj = 0; jj < L; ++jj) {
+          const int lp = (l + jj) % L;
+          store_item<D, true>(a.ptr.out[g * L + lp], lo + qidx[2 * k] / 2, a.n, v);
+        }
+      }
+    }
+  }
+}
+
 // Standalone reduce-scatter [NVRAR phase 1 over one group]: rank p writes
 // elements [p*m, (p+1)*m) of the ascending-rank sum into out[p], m = n / P.
 // Needs no flags. 16-byte path when m is a multiple of the item size (so

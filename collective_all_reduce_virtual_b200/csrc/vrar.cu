@@ -27,6 +27,7 @@ struct Settings {
   std::atomic<uint32_t> fault_mask{0};
   std::atomic<int> spin_stats{0};
   std::atomic<int> max_ctas{0};  // grid cap per call, 0 = none
+  std::atomic<int> payload_wire{VRAR_WIRE_ELEMENT};
 };
 Settings g_set;
 
@@ -159,13 +160,22 @@ int check_shape(vrar_algo_t algo, int P, int L) {
   }
 }
 
-// Payload-slot bytes (RD / HIER): P ranks x steps x items-per-slot x 32 bytes.
+// fp32 partials on the wire apply to recursive doubling and the hierarchical
+// algorithm with 16-bit elements (for fp32 elements both wires are the same).
+bool wide_wire(vrar_algo_t algo, vrar_dtype_t dt) {
+  return g_set.payload_wire.load() == VRAR_WIRE_FP32 && dt != VRAR_FP32 &&
+         (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER);
+}
+
+// Payload-slot bytes (RD / HIER): P ranks x steps x items-per-slot x 32 bytes,
+// twice that with fp32 partials of 16-bit elements (two quads per item).
 size_t ll_bytes_for(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L) {
   const int64_t items = (static_cast<int64_t>(n) + per_item(dt) - 1) / per_item(dt);
-  if (algo == VRAR_ALGO_RD) return static_cast<size_t>(P) * ilog2(P) * items * 32;
+  const size_t wide = wide_wire(algo, dt) ? 2 : 1;
+  if (algo == VRAR_ALGO_RD) return wide * static_cast<size_t>(P) * ilog2(P) * items * 32;
   if (algo == VRAR_ALGO_HIER) {
     const int64_t piece = (items + L - 1) / L;
-    return static_cast<size_t>(P) * ilog2(P / L) * piece * 32;
+    return wide * static_cast<size_t>(P) * ilog2(P / L) * piece * 32;
   }
   return 0;
 }
@@ -374,6 +384,27 @@ KernelFn staged_kernel_dt(vrar_dtype_t dt, int ti) {
                                                                       : staged_kernel<F32T>(ti);
 }
 
+template <class D>
+KernelFn pick_wide(vrar_algo_t algo, int C) {
+  if (algo == VRAR_ALGO_RD) return C <= 1 ? k_rd_wide<D, 1> : k_rd_wide<D, 2>;
+  return C <= 1 ? k_hier_wide<D, 1> : k_hier_wide<D, 2>;
+}
+
+KernelFn pick_wide_dt(vrar_dtype_t dt, vrar_algo_t algo, int C) {
+  return dt == VRAR_BF16 ? pick_wide<Bf16T>(algo, C) : pick_wide<F16T>(algo, C);
+}
+
+// Chunk count for the fp32-wire kernels (at most 2, see k_rd_wide), chosen
+// like rd_chunks_for.
+int wide_chunks_for(vrar_dtype_t dt, vrar_algo_t algo, int C, int64_t work, int P, int dev, int sms) {
+  C = std::min(C, 2);
+  for (int c = 1; c < C; ++c) {
+    const int cap = std::max(1, std::min(grid_budget(pick_wide_dt(dt, algo, c), dev, sms), kMaxCtas) / P);
+    if ((work + c - 1) / c <= static_cast<int64_t>(cap) * kThreads) return c;
+  }
+  return C;
+}
+
 int rd_chunks_for_dt(vrar_dtype_t dt, vrar_algo_t algo, int C, int64_t work, int P, int dev, int sms) {
   return dt == VRAR_BF16   ? rd_chunks_for<Bf16T>(algo, C, work, P, dev, sms)
          : dt == VRAR_FP16 ? rd_chunks_for<F16T>(algo, C, work, P, dev, sms)
@@ -436,12 +467,14 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   if ((rc = ensure_workspace(dev, ll_bytes_for(algo, P, n, dtype, L), &ws)) != VRAR_OK) return rc;
 
   int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
+  const bool wide = wide_wire(algo, dtype);
   if (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER) {
     const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
     const int64_t work = algo == VRAR_ALGO_RD ? items : (items + L - 1) / L;
-    C = rd_chunks_for_dt(dtype, algo, C, work, P, dev, ws->sms);
+    C = wide ? wide_chunks_for(dtype, algo, C, work, P, dev, ws->sms)
+             : rd_chunks_for_dt(dtype, algo, C, work, P, dev, ws->sms);
   }
-  KernelFn fn = pick_kernel_dt(dtype, algo, C);
+  KernelFn fn = wide ? pick_wide_dt(dtype, algo, C) : pick_kernel_dt(dtype, algo, C);
   if (!fn) return VRAR_EINVAL;
 
   KArgs a;
@@ -647,6 +680,13 @@ int vrar_set_max_ctas(int n) {
 }
 int vrar_get_max_ctas(void) { return g_set.max_ctas.load(); }
 
+int vrar_set_payload_wire(int wire) {
+  if (wire != VRAR_WIRE_ELEMENT && wire != VRAR_WIRE_FP32) return VRAR_EINVAL;
+  g_set.payload_wire = wire;
+  return VRAR_OK;
+}
+int vrar_get_payload_wire(void) { return g_set.payload_wire.load(); }
+
 int vrar_set_spin_stats(int on) {
   g_set.spin_stats = on ? 1 : 0;
   return VRAR_OK;
@@ -757,8 +797,10 @@ extern "C" int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* cons
   if ((rc = noalloc_setup(dev, &d)) != VRAR_OK) return rc;
 
   int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
-  C = rd_chunks_for_dt(dtype, VRAR_ALGO_RD, C, items, P, dev, d->sms);
-  KernelFn fn = pick_kernel_dt(dtype, VRAR_ALGO_RD, C);
+  const bool wide = wide_wire(VRAR_ALGO_RD, dtype);
+  C = wide ? wide_chunks_for(dtype, VRAR_ALGO_RD, C, items, P, dev, d->sms)
+           : rd_chunks_for_dt(dtype, VRAR_ALGO_RD, C, items, P, dev, d->sms);
+  KernelFn fn = wide ? pick_wide_dt(dtype, VRAR_ALGO_RD, C) : pick_kernel_dt(dtype, VRAR_ALGO_RD, C);
   KArgs a;
   std::memset(&a, 0, sizeof(a));
   for (int p = 0; p < P; ++p) {

@@ -113,7 +113,8 @@ enum {
  *     this library's choice, the page fixes none).
  *   RD (P = 2^m): m steps; at step k rank p adds its partner p XOR 2^k's
  *     current partial to its own and rounds to the element type
- *     ([NVRAR] phase 2, "Fused Payloads").
+ *     ([NVRAR] phase 2, "Fused Payloads"); with VRAR_WIRE_FP32 the partials
+ *     stay fp32 and are rounded once at the end.
  *   HIER (P = G*L, rank r = g*L + l): ascending sum over the L ranks of group
  *     g, one rounding; then RD across the G groups; then copy to the group
  *     ([NVRAR] phases 1-3). L is set by vrar_set_group_size.
@@ -161,6 +162,17 @@ VRAR_API int vrar_get_group_size(void);
  * Results do not depend on C. Range 1..8. */
 VRAR_API int vrar_set_rd_chunks(int C);
 VRAR_API int vrar_get_rd_chunks(void);
+
+/* What the fused payload words of RD and HIER carry ([NVRAR] "Fused
+ * Payloads" does not say): VRAR_WIRE_ELEMENT (default) - the partial in the
+ * element type, rounded at every step (2 bf16 / fp16 or 1 fp32 per word);
+ * VRAR_WIRE_FP32 - the fp32 partial, rounded once at the end (1 float per
+ * word: twice the words for bf16 / fp16, fewer roundings). For fp32 elements
+ * the two are the same. The in-group sum of HIER is kept in fp32 too.
+ * Process-wide setting; VRAR_EINVAL for other values. */
+enum { VRAR_WIRE_ELEMENT = 0, VRAR_WIRE_FP32 = 1 };
+VRAR_API int vrar_set_payload_wire(int wire);
+VRAR_API int vrar_get_payload_wire(void);
 
 /* Whether ONESHOT / TWOSTAGE / TWOSTAGE_WRITE run the start and end flag
  * barriers of [CAR] (default 0 = no). Across devices they keep a rank from
@@ -241,7 +253,8 @@ VRAR_API int vrar_debug_set_fault_mask(uint32_t mask);
  * library, which every GPU that loads the library holds until the process
  * exits. It calls no cudaMalloc, no cudaFree and no allocating library routine.
  *  - Limit: P must be a power of two and
- *      256 + P * log2(P) * ceil(n / e) * 32 <= VRAR_NOALLOC_SCRATCH_BYTES,
+ *      256 + P * log2(P) * ceil(n / e) * 32 * w <= VRAR_NOALLOC_SCRATCH_BYTES
+ *    (w = 2 with VRAR_WIRE_FP32 and 16-bit elements, else 1),
  *    e = 8 for bf16 / fp16, 4 for fp32 (P = 8, bf16: n <= 174,760). Larger
  *    requests return VRAR_ETOOBIG before anything is queued.
  *  - The first call on a device sets that device up: it looks up the array's

@@ -21,7 +21,7 @@ import numpy as np
 
 from . import build as _build
 
-ALGOS = ("oneshot", "twostage", "twostage_write", "rd", "hier")
+ALGOS = ("oneshot", "twostage", "twostage_write", "rd", "hier", "rd_fp32wire", "hier_fp32wire")
 _NP = {"bf16": np.uint16, "fp16": np.uint16, "fp32": np.float32}
 
 

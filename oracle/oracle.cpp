@@ -31,7 +31,10 @@
  *    ascending rank order starting from rank 0, and rounds once to the tensor
  *    type at the end.
  *  - Recursive doubling moves values in the tensor type: each step adds two
- *    tensor-typed values in fp32 and rounds back to the tensor type.
+ *    tensor-typed values in fp32 and rounds back to the tensor type. The
+ *    "fp32 wire" variants ("rd_fp32wire", "hier_fp32wire") move fp32 partials
+ *    instead: no rounding until the final store (the other reading of what a
+ *    fused payload word carries).
  *  - fp32 -> bf16 is round-to-nearest-even from the definition of the format
  *    (bf16 = the upper 16 bits of a binary32); any NaN becomes 0x7FC0.
  *  - fp32 -> fp16 is round-to-nearest-even from the definition of binary16
@@ -198,6 +201,14 @@ typename E::T reduce_ranks(const void* const* in, int first, int count, int64_t 
     return E::narrow(acc);
 }
 
+/* Same sum, kept in fp32 (no rounding): the fp32-wire variants. */
+template <class E>
+float reduce_ranks_f32(const void* const* in, int first, int count, int64_t i) {
+    float acc = E::widen(in_ptr<E>(in, first)[i]);
+    for (int q = first + 1; q < first + count; ++q) acc = add32(acc, E::widen(in_ptr<E>(in, q)[i]));
+    return acc;
+}
+
 /* One-shot [CAR]: every rank reads all P inputs and reduces the whole vector
  * into its own output. */
 template <class E>
@@ -271,6 +282,43 @@ void rd_allreduce(const void* const* in, void* const* out, int P, int64_t n, int
     recursive_doubling<E>(v, 0, n, chunks);
     for (int p = 0; p < P; ++p)
         for (int64_t i = 0; i < n; ++i) out_ptr<E>(out, p)[i] = v[p][i];
+}
+
+/* Flat recursive doubling with fp32 partials on the wire: the partials are
+ * widened once, every step adds in fp32 without rounding (the same exchange
+ * as above on fp32 buffers), and each rank rounds its result once at the end. */
+template <class E>
+void rd_allreduce_fp32wire(const void* const* in, void* const* out, int P, int64_t n, int chunks) {
+    std::vector<Buf<F32>> v(P, Buf<F32>(n));
+    for (int p = 0; p < P; ++p)
+        for (int64_t i = 0; i < n; ++i) v[p][i] = E::widen(in_ptr<E>(in, p)[i]);
+    recursive_doubling<F32>(v, 0, n, chunks);
+    for (int p = 0; p < P; ++p)
+        for (int64_t i = 0; i < n; ++i) out_ptr<E>(out, p)[i] = E::narrow(v[p][i]);
+}
+
+/* Hierarchical all-reduce with fp32 partials: the in-group sum is kept in
+ * fp32, recursive doubling across groups adds in fp32, and the all-gather
+ * stores the one rounding to the tensor type. */
+template <class E>
+void hier_allreduce_fp32wire(const void* const* in, void* const* out, int P, int64_t n, int L, int chunks) {
+    const int G = P / L;
+    Split s(n, L, E::bytes);
+    std::vector<Buf<F32>> part(P, Buf<F32>(n));
+    for (int g = 0; g < G; ++g)
+        for (int l = 0; l < L; ++l)
+            for (int64_t i = s.lo(l); i < s.hi(l); ++i) part[g * L + l][i] = reduce_ranks_f32<E>(in, g * L, L, i);
+    for (int l = 0; l < L; ++l) {
+        std::vector<Buf<F32>> across(G);
+        for (int g = 0; g < G; ++g) across[g].swap(part[g * L + l]);
+        recursive_doubling<F32>(across, s.lo(l), s.hi(l), chunks);
+        for (int g = 0; g < G; ++g) across[g].swap(part[g * L + l]);
+    }
+    for (int g = 0; g < G; ++g)
+        for (int l = 0; l < L; ++l)
+            for (int lp = 0; lp < L; ++lp)
+                for (int64_t i = s.lo(l); i < s.hi(l); ++i)
+                    out_ptr<E>(out, g * L + lp)[i] = E::narrow(part[g * L + l][i]);
 }
 
 /* Hierarchical all-reduce [NVRAR]: P = G * L ranks in G groups of L, rank
@@ -351,6 +399,16 @@ int allreduce_t(const char* algo, const void* const* in, void* const* out, int P
         hier_allreduce<E>(in, out, P, n, L, chunks);
         return 0;
     }
+    if (std::strcmp(algo, "rd_fp32wire") == 0) {
+        if (!is_pow2(P)) return -2;
+        rd_allreduce_fp32wire<E>(in, out, P, n, chunks);
+        return 0;
+    }
+    if (std::strcmp(algo, "hier_fp32wire") == 0) {
+        if (L < 1 || P % L != 0 || !is_pow2(P / L)) return -2;
+        hier_allreduce_fp32wire<E>(in, out, P, n, L, chunks);
+        return 0;
+    }
     return -1;
 }
 
@@ -382,7 +440,7 @@ void oracle_fp16_widen(const uint16_t* x, float* y, int64_t n) {
 }
 
 /* All-reduce of P rank buffers of n elements. algo: "oneshot", "twostage",
- * "twostage_write", "rd", "hier"; dtype: "bf16" or "fp16" (uint16 bit
+ * "twostage_write", "rd", "hier", "rd_fp32wire", "hier_fp32wire"; dtype: "bf16" or "fp16" (uint16 bit
  * patterns) or "fp32". L is the group size for "hier"; chunks is the chunk
  * count of the recursive-doubling phase. Returns 0, -1 (bad argument) or -2 (P/L shape the
  * algorithm does not define). */

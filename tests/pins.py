@@ -43,10 +43,10 @@ def _algos_for(P):
     """(algo, L) pairs defined for P ranks."""
     out = [("oneshot", 8), ("twostage", 8), ("twostage_write", 8)]
     if P & (P - 1) == 0:
-        out.append(("rd", 8))
+        out += [("rd", 8), ("rd_fp32wire", 8)]
         L = 1
         while L <= P:
-            out.append(("hier", L))
+            out += [("hier", L), ("hier_fp32wire", L)]
             L *= 2
     return out
 
@@ -241,6 +241,15 @@ def pin_invariants(o):
                 assert _all_equal(outs) and (bits_of(outs[0]) == bits_of(rd[0][0])).all(), "rd depends on chunks"
             assert (bits_of(o.allreduce("hier", xs, dtype, L=P)[0]) == bits_of(one[0])).all(), "hier G=1 != oneshot"
             assert (bits_of(o.allreduce("hier", xs, dtype, L=1)[0]) == bits_of(rd[0][0])).all(), "hier L=1 != rd"
+            rd32 = o.allreduce("rd_fp32wire", xs, dtype)
+            assert _all_equal(rd32)
+            assert (bits_of(o.allreduce("hier_fp32wire", xs, dtype, L=1)[0]) == bits_of(rd32[0])).all()
+            assert (bits_of(o.allreduce("hier_fp32wire", xs, dtype, L=P)[0]) == bits_of(one[0])).all(), \
+                "one group with fp32 partials is the one-shot fold"
+            if dtype == "fp32":
+                assert (bits_of(rd32[0]) == bits_of(rd[0][0])).all(), "fp32 elements: the wires agree"
+            if P <= 2:
+                assert (bits_of(rd32[0]) == bits_of(one[0])).all(), "P<=2: one add, one rounding"
             if P <= 2:
                 assert (bits_of(rd[0][0]) == bits_of(one[0])).all(), "P<=2: rd != oneshot"
             if P == 1:

@@ -157,6 +157,24 @@ def test_selector_table_entries():
     assert vrar.select_algo(8, 524288, torch.float16) == "twostage_write"
 
 
+def test_payload_wire_setting():
+    assert vrar.get_payload_wire() == "element"
+    assert L.vrar_set_payload_wire(7) == vrar.EINVAL
+    vrar.set_payload_wire("fp32")
+    try:
+        assert vrar.get_payload_wire() == "fp32"
+        # fp32 partials of bf16: twice the slot bytes; fp32 elements unchanged; one-shot needs none
+        assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 2 * 8 * 3 * 131072 * 32
+        assert vrar.workspace_bytes(8, 1 << 20, torch.float32, "rd") == 8 * 3 * 262144 * 32
+        assert vrar.workspace_bytes(32, 1 << 20, torch.float16, "hier") == 2 * 32 * 2 * 16384 * 32
+        assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "oneshot") == 0
+        # the allocation-free entry point's limit halves for bf16 with fp32 partials
+        f = L.vrar_allreduce_rd_noalloc
+        assert f(_ptrs(IN, 8), _ptrs(OUT, 8), 8, 87_380 + 8, 0, None) == vrar.ETOOBIG
+    finally:
+        vrar.set_payload_wire("element")
+
+
 def test_workspace_bytes():
     # RD at P=8 on 2 MiB of bf16 per rank: 8 ranks x 3 steps x 131072 items x 32 bytes
     assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 8 * 3 * 131072 * 32

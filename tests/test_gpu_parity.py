@@ -36,6 +36,7 @@ def _defaults():
         vrar.set_spin_timeout_ns(2_000_000_000)
         vrar.debug_set_fault_mask(0)
         vrar.set_max_ctas(0)
+        vrar.set_payload_wire("element")
 
 
 def _dev(xs_np, dtype):
@@ -43,10 +44,14 @@ def _dev(xs_np, dtype):
 
 
 def run(algo, xs_np, dtype, L=8, C=4, edge=False):
+    """One call through the binding. 'rd_fp32wire' / 'hier_fp32wire' are the
+    oracle's names for RD / HIER with fp32 partials on the wire."""
     vrar.set_group_size(L)
     vrar.set_rd_chunks(C)
     vrar.set_edge_sync(edge)
-    outs = vrar.all_reduce(_dev(xs_np, dtype), algo=algo)
+    wire = algo.endswith("_fp32wire")
+    vrar.set_payload_wire("fp32" if wire else "element")
+    outs = vrar.all_reduce(_dev(xs_np, dtype), algo=algo[: -len("_fp32wire")] if wire else algo)
     rc, info = vrar.query_status()
     assert rc == 0, f"device status {rc} {info}"
     return [to_np(o) for o in outs]
@@ -62,9 +67,9 @@ def assert_bits(got, want, what):
 def algos_for(P):
     out = [("oneshot", 8), ("twostage", 8), ("twostage_write", 8)]
     if P & (P - 1) == 0:
-        out.append(("rd", 8))
+        out += [("rd", 8), ("rd_fp32wire", 8)]
         for L in sorted({1, max(1, P // 2), P}):
-            out.append(("hier", L))
+            out += [("hier", L), ("hier_fp32wire", L)]
     return out
 
 
@@ -420,6 +425,7 @@ def test_spin_stats_count_timeouts():
 # ---- failure detection: bounded waits, no GPU fault ----------------------------------------------
 
 @pytest.mark.parametrize("algo,P,L,edge,phase", [
+    ("rd_fp32wire", 4, 8, True, 4),
     ("oneshot", 4, 8, True, 1),
     ("twostage", 4, 8, False, 2),
     ("twostage_write", 8, 8, True, 1),
@@ -434,13 +440,16 @@ def test_missing_rank_times_out_and_recovers(algo, P, L, edge, phase):
     vrar.set_group_size(L)
     vrar.set_edge_sync(edge)
     vrar.set_spin_timeout_ns(50_000_000)
+    wire = algo.endswith("_fp32wire")
+    vrar.set_payload_wire("fp32" if wire else "element")
+    base = algo[: -len("_fp32wire")] if wire else algo
     vrar.debug_set_fault_mask(1 << 1)
-    vrar.all_reduce(d_in, algo=algo)
+    vrar.all_reduce(d_in, algo=base)
     rc, info = vrar.query_status()
     assert rc == vrar.ETIMEDOUT, (rc, info)
     assert info[1] == phase
     vrar.debug_set_fault_mask(0)
-    outs = vrar.all_reduce(d_in, algo=algo)
+    outs = vrar.all_reduce(d_in, algo=base)
     rc, info = vrar.query_status()
     assert rc == 0, info
     assert_bits([to_np(o) for o in outs], oracle.allreduce(algo, xs, "bf16", L=L), f"{algo} after timeout")

@@ -45,6 +45,9 @@ MUTANTS = {
                              "if (rest >= 0x1000u) keep += 1;"),
     "half_subnormal_truncate": ("if (rest > 0.5f || (rest == 0.5f && (i & 1u))) i += 1;",
                                 "if (rest > 2.0f) i += 1;"),
+    "fp32wire_hier_rounds_group_sum": (
+        "part[g * L + l][i] = reduce_ranks_f32<E>(in, g * L, L, i);",
+        "part[g * L + l][i] = E::widen(reduce_ranks<E>(in, g * L, L, i));"),
     "half_widen_bias": ("return bits_to_f32(sign | ((exp + 112u) << 23) | (frac << 13));",
                         "return bits_to_f32(sign | ((exp + 111u) << 23) | (frac << 13));"),
 }

@@ -23,19 +23,23 @@ if torch.cuda.is_available():
 else:  # collected on the CPU machine, never run there
     vrar = None
 
-RTOL = {"bf16": 1e-2, "fp32": 1e-5}
-DT = {"bf16": 0, "fp32": 1}
+RTOL = {"bf16": 1e-2, "fp32": 1e-5, "fp16": 5e-3}
+DT = {"bf16": 0, "fp32": 1, "fp16": 2}
 
-# (P, n, dtype): a tiny ragged case, the P=2 128 KiB shape, a several-CTA
+# (P, n, dtype, wire): a tiny ragged case, the P=2 128 KiB shape, a several-CTA
 # ragged case, and the largest request the fixed scratch holds at P = 8
-# (8 * 3 * ceil(n / e) * 32 + 256 <= 16 MiB: n <= 174,760 bf16, 87,380 fp32).
-CASES = [(4, 7, "bf16"), (2, 65_536, "bf16"), (8, 100_003, "bf16"), (8, 174_760, "bf16"),
-         (4, 7, "fp32"), (2, 65_536, "fp32"), (8, 50_003, "fp32"), (8, 87_380, "fp32")]
+# (8 * 3 * ceil(n / e) * 32 * w + 256 <= 16 MiB: n <= 174,760 bf16, 87,380 fp32,
+# 87,376 bf16 with fp32 partials on the wire).
+CASES = [(4, 7, "bf16", "element"), (2, 65_536, "bf16", "element"), (8, 100_003, "bf16", "element"),
+         (8, 174_760, "bf16", "element"), (4, 7, "fp32", "element"), (2, 65_536, "fp32", "element"),
+         (8, 50_003, "fp32", "element"), (8, 87_380, "fp32", "element"), (8, 50_001, "fp16", "element"),
+         (8, 87_376, "bf16", "fp32")]  # fp32 partials of bf16: twice the slot bytes per item
 
 
-@pytest.mark.parametrize("P,n,dtype", CASES)
-def test_noalloc_matches_allocating_rd_on_two_calls(P, n, dtype):
+@pytest.mark.parametrize("P,n,dtype,wire", CASES)
+def test_noalloc_matches_allocating_rd_on_two_calls(P, n, dtype, wire):
     lib = vrar.lib()
+    vrar.set_payload_wire(wire)
     xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=900 + P)
     d_in = [from_np(x, dtype).cuda() for x in xs]
     ref = vrar.all_reduce(d_in, algo="rd")
@@ -58,4 +62,5 @@ def test_noalloc_matches_allocating_rd_on_two_calls(P, n, dtype):
             assert np.array_equal(bits_of(got), bits_of(ref_np[p])), f"call {call} rank {p}"
             y = oracle.to_float(got, dtype)
             assert (np.abs(y - S) <= RTOL[dtype] * A).all(), f"call {call} rank {p}: tolerance"
+    vrar.set_payload_wire("element")
 
