@@ -66,6 +66,12 @@ SWEEP = (
     + [dict(name=f"P=32 hier 4x8 {b >> 10} KiB per rank, uniform(-1,1)", P=32, n=b // 2, dtype="bf16",
             dist="uniform:-1,1", L=8, algos=("hier", "oneshot", "twostage_write", "auto")) for b in
        (256 << 10, 2 << 20)]
+    + [dict(name=f"P=8 fp16 {b >> 10} KiB per rank, N(0,1)", P=8, n=b // 2, dtype="fp16", dist="normal:0,1",
+            algos=("oneshot", "twostage_write", "rd", "auto")) for b in (1 << 20, 2 << 20)]
+    + [dict(name=f"P=8 bf16 {b >> 10} KiB per rank, N(0,1), RD with fp32 partials on the wire", P=8, n=b // 2,
+            dtype="bf16", dist="normal:0,1", algos=("rd",), wire="fp32") for b in (128 << 10, 2 << 20)]
+    + [dict(name="P=32 hier 4x8 2048 KiB per rank, uniform(-1,1), fp32 partials on the wire", P=32,
+            n=(2 << 20) // 2, dtype="bf16", dist="uniform:-1,1", L=8, algos=("hier",), wire="fp32")]
     + [dict(name="P=8 prefill 16384x7168 bf16 (224 MiB per rank), N(0,0.02)", P=8, n=16384 * 7168,
             dtype="bf16", dist="normal:0,0.02", algos=("twostage", "twostage_write", "auto"), steps=20,
             collectives=("rs", "ag"))]
@@ -76,8 +82,8 @@ SWEEP = (
 # share one order, so any of them gives the same bits).
 REFERENCE_ALGO = "twostage_write"
 
-TDT = {"bf16": torch.bfloat16, "fp32": torch.float32}
-ESZ = {"bf16": 2, "fp32": 4}
+TDT = {"bf16": torch.bfloat16, "fp32": torch.float32, "fp16": torch.float16}
+ESZ = {"bf16": 2, "fp32": 4, "fp16": 2}
 
 
 # ---- small helpers (host logic; tested on the CPU) ---------------------------------------------
@@ -360,35 +366,64 @@ def entry(wl: Workload, t_s: float, peak: float):
 
 
 def measure_e2e(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None):
-    """Inputs copied from pinned host memory, all-reduce, outputs copied back:
-    every step, inside the timed region (eager calls through the binding)."""
+    """Every step copies its P inputs from pinned host memory to the device,
+    runs the all-reduce through the public binding, and copies its P outputs
+    back to pinned host memory. Steps are pipelined the way a user streaming
+    batches would: copies in (one stream), the all-reduce (another) and copies
+    out (a third) of consecutive steps overlap, on two device buffer sets; PCIe
+    carries both directions at once."""
     vrar = wl.vrar
-    h_in = [t.cpu().pin_memory() for t in wl.base]
-    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.base]
-    d_in, d_out = wl.ins[0], wl.outs[0]
+    # The P rank buffers of a set are rows of one [P, n] block, so that a step
+    # moves its inputs in one copy and its outputs out in one copy.
+    dev = wl.base[0].device
+    h_in = torch.stack([t.cpu() for t in wl.base]).pin_memory()
+    h_out = [torch.empty_like(h_in).pin_memory() for _ in range(2)]
+    sets = 2
+    d_in_blk = [torch.empty(h_in.shape, dtype=h_in.dtype, device=dev) for _ in range(sets)]
+    d_out_blk = [torch.empty(h_in.shape, dtype=h_in.dtype, device=dev) for _ in range(sets)]
+    d_in = [list(blk.unbind(0)) for blk in d_in_blk]
+    d_out = [list(blk.unbind(0)) for blk in d_out_blk]
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    run_done = [ev(), ev()]
+    out_done = [ev(), ev()]
+    for e in run_done + out_done:
+        e.record(torch.cuda.current_stream())
 
-    def step():
-        for d, h in zip(d_in, h_in):
-            d.copy_(h, non_blocking=True)
-        vrar.all_reduce(d_in, d_out, algo=algo)
-        for h, d in zip(h_out, d_out):
-            h.copy_(d, non_blocking=True)
+    def step(i):
+        b = i % sets
+        s_in.wait_event(run_done[b])          # the step two back has read these inputs
+        with torch.cuda.stream(s_in):
+            d_in_blk[b].copy_(h_in, non_blocking=True)
+        in_done = ev()
+        in_done.record(s_in)
+        s_run.wait_event(in_done)
+        s_run.wait_event(out_done[b])         # the step two back has copied these outputs out
+        vrar.all_reduce(d_in[b], d_out[b], algo=algo, stream=s_run)
+        run_done[b].record(s_run)
+        s_out.wait_event(run_done[b])
+        with torch.cuda.stream(s_out):
+            h_out[b].copy_(d_out_blk[b], non_blocking=True)
+        out_done[b].record(s_out)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
-    s = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, device)
-    e0.record(s)
-    for _ in range(steps):
-        step()
-    e1.record(s)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(steps):
+        step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_run)
+    e1.record(s_out)
     e1.synchronize()
+    torch.cuda.synchronize()
     barrier(world, device)
     ms = max_over_ranks(e0.elapsed_time(e1), world, device) / steps
-    bytes_in = sum(t.numel() * t.element_size() for t in h_in)
-    bytes_out = sum(t.numel() * t.element_size() for t in h_out)
+    bytes_in = h_in.numel() * h_in.element_size()
+    bytes_out = h_out[0].numel() * h_out[0].element_size()
+    del d_in_blk, d_out_blk
     return ms, bytes_in, bytes_out
 
 
@@ -454,6 +489,7 @@ def run_vrar(args):
         for spec in SWEEP:
             if spec.get("L"):
                 vrar.set_group_size(spec["L"])
+            vrar.set_payload_wire(spec.get("wire", "element"))
             w = Workload(spec, device)
             row = {"workload": spec["name"], "P": w.P, "n": w.n, "rotating_sets": w.R,
                    "selected": vrar.select_algo(w.P, w.n, TDT[w.dt])}
@@ -469,6 +505,9 @@ def run_vrar(args):
             w.free()
             torch.cuda.empty_cache()
             vrar.set_group_size(8)
+            vrar.set_payload_wire("element")
+            if "wire" in spec:
+                row["wire"] = spec["wire"]
             sweep.append(row)
     clk = clocks.stop()
 
