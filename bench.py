@@ -256,6 +256,7 @@ class Workload:
         self.out_arr = [vrar.ptr_array([t.data_ptr() for t in s]) for s in self.outs]
         self.lib = vrar.lib()
         self.dtc = vrar.DTYPES[TDT[self.dt]]
+        self.small = None
 
     def call(self, i: int, algo: str, stream_handle: int):
         r = i % self.R
@@ -272,8 +273,26 @@ class Workload:
                 self.call(offset + i, algo, h)
         return g
 
+    def collective_call(self, i: int, kind: str, stream_handle: int):
+        """Standalone reduce-scatter ('rs': inputs -> n/P slices) or all-gather
+        ('ag': n/P slices -> outputs) on this workload's buffer set i % R."""
+        if self.small is None:
+            m = self.n // self.P
+            self.small = [[torch.empty(m, dtype=self.base[0].dtype, device=self.base[0].device)
+                           for _ in range(self.P)] for _ in range(self.R)]
+            self.small_arr = [self.vrar.ptr_array([t.data_ptr() for t in s]) for s in self.small]
+        r = i % self.R
+        if kind == "rs":
+            rc = self.lib.vrar_reduce_scatter(self.in_arr[r], self.small_arr[r], self.P, self.n, self.dtc,
+                                              stream_handle)
+        else:
+            rc = self.lib.vrar_all_gather(self.small_arr[r], self.out_arr[r], self.P, self.n, self.dtc,
+                                          stream_handle)
+        if rc != 0:
+            raise self.vrar.VrarError(rc, kind)
+
     def free(self):
-        self.ins = self.outs = self.base = None
+        self.ins = self.outs = self.base = self.small = None
 
 
 def upload_graph(g) -> bool:
@@ -323,23 +342,7 @@ def measure_algo(wl: Workload, algo: str, steps: int, warmup: int, world=1, devi
 def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1, device=None):
     """Milliseconds per call of the standalone reduce-scatter ('rs') or
     all-gather ('ag') on the workload's shape (graph of `steps` calls)."""
-    vrar = wl.vrar
-    lib, P, n = wl.lib, wl.P, wl.n
-    m = n // P
-    small = [[torch.empty(m, dtype=wl.base[0].dtype, device=wl.base[0].device) for _ in range(P)]
-             for _ in range(wl.R)]
-    small_arr = [vrar.ptr_array([t.data_ptr() for t in s]) for s in small]
-
-    def call(i, h):
-        r = i % wl.R
-        if kind == "rs":
-            rc = lib.vrar_reduce_scatter(wl.in_arr[r], small_arr[r], P, n, wl.dtc, h)
-        else:
-            rc = lib.vrar_all_gather(small_arr[r], wl.out_arr[r], P, n, wl.dtc, h)
-        if rc != 0:
-            raise vrar.VrarError(rc, kind)
-
-    call(0, torch.cuda.current_stream().cuda_stream)
+    wl.collective_call(0, kind, torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
 
     def graph(count, offset):
@@ -347,14 +350,14 @@ def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1
         with torch.cuda.graph(g):
             h = torch.cuda.current_stream().cuda_stream
             for i in range(count):
-                call(offset + i, h)
+                wl.collective_call(offset + i, kind, h)
         return g
 
     gw, gt = graph(warmup, 0), graph(steps, warmup)
     gw.replay()
     torch.cuda.synchronize()
     ms = max_over_ranks(time_graph(gt, world, device), world, device)
-    del gw, gt, small
+    del gw, gt
     return ms / steps
 
 
@@ -606,7 +609,9 @@ def run_selector_sweep(args):
 
 def run_case(spec_text: str):
     """A few back-to-back calls of one algorithm on one shape (for profilers):
-    'algo,P,KiB[,calls]'. Exits non-zero if the device status is not clean."""
+    'algo,P,KiB[,calls]', algo an all-reduce algorithm or 'rs' / 'ag' (the
+    standalone reduce-scatter / all-gather; KiB is the full per-rank vector).
+    Exits non-zero if the device status is not clean."""
     import collective_all_reduce_virtual_b200 as vrar
     parts = spec_text.split(",")
     algo, P, kib = parts[0], int(parts[1]), int(parts[2])
@@ -616,7 +621,10 @@ def run_case(spec_text: str):
     wl = Workload(dict(WORKLOAD, P=P, n=kib * 512, name=spec_text), device)
     h = torch.cuda.current_stream().cuda_stream
     for i in range(calls):
-        wl.call(i, algo, h)
+        if algo in ("rs", "ag"):
+            wl.collective_call(i, algo, h)
+        else:
+            wl.call(i, algo, h)
     torch.cuda.synchronize()
     rc, info = vrar.query_status()
     print(json.dumps({"case": spec_text, "status": rc, "info": info}))
