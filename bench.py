@@ -495,7 +495,8 @@ def run_vrar(args):
             vrar.set_payload_wire(spec.get("wire", "element"))
             w = Workload(spec, device)
             row = {"workload": spec["name"], "P": w.P, "n": w.n, "rotating_sets": w.R,
-                   "selected": vrar.select_algo(w.P, w.n, TDT[w.dt])}
+                   "selected": vrar.select_algo(w.P, w.n, TDT[w.dt]),
+                   "kernel": vrar.kernel_name(w.P, w.n, TDT[w.dt], "auto")}
             for algo in spec["algos"]:
                 k = spec.get("steps", 200)
                 row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device) / 1e3, peak)
@@ -517,8 +518,7 @@ def run_vrar(args):
     P, n, esz = WORKLOAD["P"], WORKLOAD["n"], ESZ[WORKLOAD["dtype"]]
     value = world * busbw_gbs(P, n, esz, t_s)
     achieved = b_min_bytes(P, n, esz) / t_s / 1e9
-    kernel = {"oneshot": "k_oneshot", "twostage": "k_twostage", "twostage_write": "k_twostage_write",
-              "rd": "k_rd", "hier": "k_hier"}[algo_auto]
+    kernel = vrar.kernel_name(P, n, TDT[WORKLOAD["dtype"]], "auto")
     traffic, traffic_src = profiled_traffic(kernel, "decode_p8_1mib")
 
     line = {
@@ -586,7 +586,8 @@ def run_reference(args):
 def run_selector_sweep(args):
     """Every algorithm at every (P, bytes per rank) of the selector table, as
     JSON lines (one per shape). The write-mode kernel is the one this process
-    runs (VRAR_WRITE_KERNEL=plain|staged forces one)."""
+    runs (VRAR_WRITE_KERNEL=plain|staged|async forces one; with staged or
+    async only the write mode is timed)."""
     import collective_all_reduce_virtual_b200 as vrar
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
@@ -595,9 +596,11 @@ def run_selector_sweep(args):
         for kib in (32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384):
             spec = dict(WORKLOAD, P=P, n=kib * 512, name=f"P={P} {kib} KiB per rank")
             wl = Workload(spec, device)
-            row = {"P": P, "kib": kib, "write_kernel": kernel, "selected": vrar.select_algo(P, wl.n, TDT[wl.dt])}
+            row = {"P": P, "kib": kib, "write_kernel": kernel, "selected": vrar.select_algo(P, wl.n, TDT[wl.dt]),
+                   "kernel": vrar.kernel_name(P, wl.n, TDT[wl.dt], "auto")}
             steps = 200 if kib <= 4096 else 50
-            algos = ("oneshot", "twostage_write", "twostage", "rd") if kernel != "staged" else ("twostage_write",)
+            algos = ("oneshot", "twostage_write", "twostage", "rd") if kernel not in ("staged", "async") \
+                else ("twostage_write",)
             for algo in algos:
                 if algo == "rd" and P & (P - 1):
                     continue

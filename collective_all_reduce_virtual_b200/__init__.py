@@ -41,6 +41,7 @@ SIGNATURES = {
     "vrar_reduce_scatter": ([_pp, _pp, _i, _sz, _i, _vp], _i),
     "vrar_all_gather": ([_pp, _pp, _i, _sz, _i, _vp], _i),
     "vrar_select_algo": ([_i, _sz, _i], _i),
+    "vrar_kernel_name": ([_i, _sz, _i, _i], ctypes.c_char_p),
     "vrar_set_group_size": ([_i], _i),
     "vrar_get_group_size": ([], _i),
     "vrar_set_rd_chunks": ([_i], _i),
@@ -176,6 +177,14 @@ def select_algo(P: int, n: int, dtype: torch.dtype = torch.bfloat16) -> str:
     return ALGO_NAMES[_check(_lib.vrar_select_algo(P, n, DTYPES[dtype]), "vrar_select_algo")]
 
 
+def kernel_name(P: int, n: int, dtype: torch.dtype = torch.bfloat16, algo: str = "auto") -> str:
+    """Base name of the kernel all_reduce(P buffers of n, dtype, algo) would launch."""
+    name = _lib.vrar_kernel_name(P, n, DTYPES[dtype], ALGOS[algo])
+    if name is None:
+        raise VrarError(EINVAL, "vrar_kernel_name")
+    return name.decode()
+
+
 def set_group_size(L: int) -> None:
     _check(_lib.vrar_set_group_size(L), "vrar_set_group_size")
 
@@ -274,7 +283,7 @@ def version() -> int:
     return _lib.vrar_version()
 
 
-__all__ = ["all_reduce", "reduce_scatter", "all_gather", "select_algo", "set_group_size",
+__all__ = ["all_reduce", "reduce_scatter", "all_gather", "select_algo", "kernel_name", "set_group_size",
            "get_group_size", "set_rd_chunks", "get_rd_chunks", "set_payload_wire", "get_payload_wire", "set_edge_sync", "get_edge_sync",
            "set_max_ctas", "get_max_ctas", "set_spin_timeout_ns", "get_spin_timeout_ns", "query_status", "reserve",
            "workspace_bytes", "reset", "set_spin_stats", "get_spin_stats", "debug_set_fault_mask", "strerror", "version", "VrarError",

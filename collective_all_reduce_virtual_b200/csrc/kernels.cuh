@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
 // r and streams it to all P outputs. The slice is cut into tiles of
 // kStageItems items; CTA b of rank r takes tiles b, b+B, b+2B, ... A producer
 // (lane 0 of warp 0) keeps up to `stages` tiles in flight: per tile, one bulk
-// copy per input rank (2 KiB each) into a shared-memory stage, completing an
+// copy per input rank (kStageItems * 16 bytes) into a shared-memory stage, completing an
 // mbarrier transaction count. Consumer warps (one thread per item) sum the P
 // copies of their item from shared memory in ascending rank order, round once,
 // and store the result to the P outputs, then free the stage for the producer.
@@ -261,6 +261,82 @@ __global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(cons
   }
   // Ragged last item, by the slice owner's first CTA.
   if (threadIdx.x == 32 && c.b == 0 && full_items < a.items && full_items >= lo && full_items < hi) {
+    const uint4 v = reduce_item<D>(a.ptr, 0, a.P, full_items, a.n);
+    for (int p = 0; p < a.P; ++p) store_item<D, true>(a.ptr.out[p], full_items, a.n, v);
+  }
+  if (a.edge_sync) {
+    __threadfence();
+    block_barrier(a, c, kPhEnd);
+  }
+}
+
+// 2-stage write mode [CAR "cross_device_reduce_2stage", write mode] with
+// per-thread asynchronous copies. Same result and work split as
+// k_twostage_write: thread i of CTA b (rank r) takes item i of tiles b, b+B,
+// ... of slice r. For each tile it issues P 16-byte async copies (one per input
+// rank) into its own shared-memory slots and keeps S tiles in flight; it then
+// sums its P slots in ascending rank order, rounds once, and stores to all P
+// outputs. A thread reads only slots it filled itself, so its own copy groups
+// are the only synchronisation: no mbarrier, no producer lane, and all TI
+// threads issue copies in parallel (the staged kernel's single producer lane
+// issues P bulk copies per tile one after another, which is what limits it
+// on small messages at many ranks). Shared memory: S * P * TI * 16 bytes.
+template <class D, int TI, int S>
+__global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const int64_t full_items = a.n / D::VE;
+  const int64_t piece = (a.items + a.P - 1) / a.P;
+  const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
+  const int64_t hi_full = hi < full_items ? hi : full_items;
+  const int64_t rank_tiles = hi_full > lo ? (hi_full - lo + TI - 1) / TI : 0;
+  const int64_t ntile = rank_tiles > c.b ? (rank_tiles - c.b + a.B - 1) / a.B : 0;
+  auto tile_base = [&](int64_t k) { return lo + (c.b + k * a.B) * TI; };
+  if (threadIdx.x < a.P) {
+    for (int64_t k = 0; k < ntile && k < S; ++k) {
+      const int64_t base = tile_base(k);
+      prefetch_items<D>(a.ptr.in[threadIdx.x], base, hi_full - base < TI ? hi_full - base : TI, a.n);
+    }
+  }
+  pdl_wait();
+  if (a.edge_sync) {
+    cta_publish_flag(c, cta_take_ticket(a));
+    if (!block_barrier(a, c, kPhStart)) return;
+  }
+  const size_t stage_bytes = static_cast<size_t>(a.P) * TI * 16;
+  unsigned char* mine = smem + threadIdx.x * 16;
+  auto issue = [&](int64_t k) {
+    if (k < ntile) {
+      const int64_t it = tile_base(k) + threadIdx.x;
+      if (it < hi_full) {
+        unsigned char* dst = mine + (k % S) * stage_bytes;
+        for (int p = 0; p < a.P; ++p)
+          cp_async16(dst + p * (TI * 16), static_cast<const unsigned char*>(a.ptr.in[p]) + it * 16);
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int k = 0; k < S - 1; ++k) issue(k);
+  for (int64_t k = 0; k < ntile; ++k) {
+    issue(k + S - 1);
+    cp_async_wait<S - 1>();
+    const int64_t it = tile_base(k) + threadIdx.x;
+    if (it < hi_full) {
+      const unsigned char* src = mine + (k % S) * stage_bytes;
+      Acc<D> acc;
+      acc.init(ld_shared_v4(src));
+      for (int p = 1; p < a.P; ++p) acc.add(ld_shared_v4(src + p * (TI * 16)));
+      const uint4 v = acc.round();
+      for (int j = 0; j < a.P; ++j) {
+        const int q = (c.r + j) % a.P;
+        st_stream(static_cast<typename D::E*>(a.ptr.out[q]) + it * D::VE, v);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  if (threadIdx.x == 0 && c.b == 0 && full_items < a.items && full_items >= lo && full_items < hi) {
     const uint4 v = reduce_item<D>(a.ptr, 0, a.P, full_items, a.n);
     for (int p = 0; p < a.P; ++p) store_item<D, true>(a.ptr.out[p], full_items, a.n, v);
   }

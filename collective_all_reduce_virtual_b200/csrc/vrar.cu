@@ -202,7 +202,9 @@ bool ensure_smem_limit(KernelFn fn, int dev, size_t smem) {
   static std::mutex mu;
   static Entry set[256];
   static int used = 0;
-  if (smem <= 48 * 1024) return true;
+  // Set for any dynamic size: the 48 KiB default covers static shared memory
+  // too, so a launch just under it can still be refused without the attribute.
+  if (smem == 0) return true;
   std::lock_guard<std::mutex> lock(mu);
   Entry* e = nullptr;
   for (int i = 0; i < used; ++i)
@@ -324,32 +326,41 @@ int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream, int threa
   return VRAR_OK;
 }
 
-// Which write-mode kernel runs: VRAR_WRITE_KERNEL=plain|staged forces one
-// (read once); otherwise write_staged_for() decides by shape.
+// Which write-mode kernel runs: VRAR_WRITE_KERNEL=plain|staged|async forces
+// one (read once); otherwise write_kernel_for() decides by shape.
+enum WriteKernel { kWritePlain = 0, kWriteStaged = 1, kWriteAsync = 2 };
+
 int write_kernel_override() {
   static int cached = -2;
   if (cached == -2) {
     const char* s = std::getenv("VRAR_WRITE_KERNEL");
-    cached = !s ? -1 : std::strcmp(s, "plain") == 0 ? 0 : std::strcmp(s, "staged") == 0 ? 1 : -1;
+    cached = !s                               ? -1
+             : std::strcmp(s, "plain") == 0  ? kWritePlain
+             : std::strcmp(s, "staged") == 0 ? kWriteStaged
+             : std::strcmp(s, "async") == 0  ? kWriteAsync
+                                             : -1;
   }
   return cached;
 }
 
 // Per-shape choice measured on a B200 (CUDA-graph timings of back-to-back
 // calls, inputs rotated through more than 3x the L2 size): 'O' one-shot,
-// 'P' write mode with the plain kernel, 'S' write mode with the shared-memory
-// staged kernel. Rows: P <= 2, 4, 8, 16, 32; columns: bytes per rank
-// <= 32 KiB, 64 KiB, ..., 8 MiB, and above. One-shot wins small messages at
-// few ranks (a single pass, its P-fold re-reads served by L2); the write mode
-// moves the minimum traffic and wins everywhere else; the staged kernel
-// overlaps tile loads with stores and wins except around 1 MiB per rank and
-// at 32 ranks above 2 MiB.
+// 'A' write mode with the per-thread async-copy kernel, 'S' write mode with
+// the bulk-copy staged kernel, 'P' write mode with the plain kernel. Rows:
+// P <= 2, 4, 8, 16, 32; columns: bytes per rank <= 32 KiB, 64 KiB, ...,
+// 8 MiB, and above. One-shot keeps small messages at two ranks (one pass,
+// its re-reads served by L2). The async write kernel wins almost everywhere
+// else: every thread keeps all P loads of its items in flight, with no
+// serial issue. From 8 MiB per rank at 4-16 ranks the bulk-copy pipeline
+// streams a little better, and at 32 ranks from 4 MiB the plain kernel
+// (shared-memory stages of 32 ranks cost occupancy); both margins are a few
+// percent.
 constexpr char kChoice[5][10] = {
-    {'O', 'O', 'O', 'O', 'O', 'O', 'O', 'S', 'S', 'S'},  // P <= 2
-    {'O', 'O', 'O', 'O', 'O', 'P', 'S', 'S', 'S', 'S'},  // P <= 4
-    {'O', 'O', 'O', 'O', 'S', 'P', 'S', 'S', 'S', 'S'},  // P <= 8
-    {'S', 'S', 'S', 'S', 'S', 'P', 'P', 'S', 'S', 'S'},  // P <= 16
-    {'S', 'S', 'S', 'S', 'S', 'P', 'S', 'P', 'P', 'P'},  // P <= 32
+    {'O', 'O', 'O', 'O', 'O', 'O', 'O', 'A', 'A', 'A'},  // P <= 2
+    {'A', 'A', 'A', 'O', 'O', 'A', 'A', 'A', 'S', 'A'},  // P <= 4
+    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 8
+    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 16
+    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'P'},  // P <= 32
 };
 
 char shape_choice(int P, size_t bytes) {
@@ -360,10 +371,48 @@ char shape_choice(int P, size_t bytes) {
   return kChoice[row][col];
 }
 
-bool write_staged_for(int P, size_t bytes) {
+// Which write-mode kernel runs a TWOSTAGE_WRITE call. Shapes the table gives
+// to one-shot (when write mode is asked for by name) take the async kernel,
+// the fastest write kernel on small messages.
+int write_kernel_for(int P, size_t bytes) {
   const int forced = write_kernel_override();
-  if (forced >= 0) return forced == 1;
-  return shape_choice(P, bytes) != 'P';
+  if (forced >= 0) return forced;
+  const char ch = shape_choice(P, bytes);
+  return ch == 'P' ? kWritePlain : ch == 'S' ? kWriteStaged : kWriteAsync;
+}
+
+// Async-copy kernel: 64 items (one per thread) per tile, and S tiles in flight
+// per thread. S is set from the bytes a CTA should keep in flight, measured:
+// small messages give each CTA only a tile or two, and they run fastest with
+// deep stages (about 192 KiB per CTA up to 64 KiB per rank, 96 KiB up to
+// 256 KiB); from 512 KiB per rank smaller CTAs, more of them per SM, do better
+// (48 KiB, then 32 KiB). With a CTA budget of at most one CTA per SM every CTA
+// keeps the deepest setting. S is rounded down to an instantiated depth
+// (3, 4, 6 or 8).
+constexpr int kAsyncTileItems = 64;
+
+int async_stages(int P, size_t bytes_per_rank, bool deep) {
+  const size_t kib = 1024;
+  const size_t target = deep || bytes_per_rank <= 64 * kib ? 192 * kib
+                        : bytes_per_rank <= 256 * kib      ? 96 * kib
+                        : bytes_per_rank <= 512 * kib      ? 48 * kib
+                                                           : 32 * kib;
+  const size_t s = target / (static_cast<size_t>(P) * kAsyncTileItems * 16);
+  return s >= 8 ? 8 : s >= 6 ? 6 : s >= 4 ? 4 : 3;
+}
+
+template <class D>
+KernelFn async_kernel(int S) {
+  switch (S) {
+    case 8: return k_twostage_write_async<D, kAsyncTileItems, 8>;
+    case 6: return k_twostage_write_async<D, kAsyncTileItems, 6>;
+    case 4: return k_twostage_write_async<D, kAsyncTileItems, 4>;
+    default: return k_twostage_write_async<D, kAsyncTileItems, 3>;
+  }
+}
+
+KernelFn async_kernel_dt(vrar_dtype_t dt, int S) {
+  return dt == VRAR_BF16 ? async_kernel<Bf16T>(S) : dt == VRAR_FP16 ? async_kernel<F16T>(S) : async_kernel<F32T>(S);
 }
 
 constexpr int kWriteTileItems = 64;  // staged write mode: items per tile (1 KiB per input rank)
@@ -513,7 +562,20 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     }
     default: break;
   }
-  if (algo == VRAR_ALGO_TWOSTAGE_WRITE && write_staged_for(P, n * elem_size(dtype))) {
+  const int wk = algo == VRAR_ALGO_TWOSTAGE_WRITE ? write_kernel_for(P, n * elem_size(dtype)) : kWritePlain;
+  if (wk == kWriteAsync) {
+    const int cap_budget = g_set.max_ctas.load();
+    const bool deep = cap_budget > 0 && cap_budget <= ws->sms;
+    const int S = async_stages(P, n * elem_size(dtype), deep);
+    KernelFn af = async_kernel_dt(dtype, S);
+    const int64_t tiles = std::max<int64_t>(1, (work + kAsyncTileItems - 1) / kAsyncTileItems);
+    const size_t smem = static_cast<size_t>(S) * P * kAsyncTileItems * 16;
+    const int resident = grid_budget(af, dev, ws->sms, kAsyncTileItems, smem);
+    if (resident < 1) return VRAR_ECUDA;
+    a.B = static_cast<int>(std::min<int64_t>(tiles, std::max(1, std::min(resident, kMaxCtas) / P)));
+    return launch(af, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), kAsyncTileItems, smem);
+  }
+  if (wk == kWriteStaged) {
     // Normally 64-item tiles and about 96 KiB of stages per CTA (two CTAs per
     // SM). When a CTA budget leaves at most one CTA per SM, each CTA must keep
     // far more bytes in flight to draw its share of memory bandwidth: 128-item
@@ -595,6 +657,27 @@ int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, 
 int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype) {
   if (P < 1 || P > kMaxRanks || !valid_dtype(dtype)) return VRAR_EINVAL;
   return select_algo(P, n, dtype);
+}
+
+const char* vrar_kernel_name(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t algo) {
+  if (P < 1 || P > kMaxRanks || !valid_dtype(dtype) || algo < VRAR_ALGO_AUTO || algo > VRAR_ALGO_HIER)
+    return nullptr;
+  if (algo == VRAR_ALGO_AUTO) {
+    const int forced = env_algo();
+    algo = static_cast<vrar_algo_t>(forced > 0 ? forced : select_algo(P, n, dtype));
+  }
+  switch (algo) {
+    case VRAR_ALGO_ONESHOT: return "k_oneshot";
+    case VRAR_ALGO_TWOSTAGE: return "k_twostage";
+    case VRAR_ALGO_TWOSTAGE_WRITE: {
+      const int wk = write_kernel_for(P, n * elem_size(dtype));
+      return wk == kWriteAsync ? "k_twostage_write_async" : wk == kWriteStaged ? "k_twostage_write_staged"
+                                                                                : "k_twostage_write";
+    }
+    case VRAR_ALGO_RD: return wide_wire(algo, dtype) ? "k_rd_wide" : "k_rd";
+    case VRAR_ALGO_HIER: return wide_wire(algo, dtype) ? "k_hier_wide" : "k_hier";
+    default: return nullptr;
+  }
 }
 
 int vrar_set_group_size(int L) {

@@ -150,6 +150,20 @@ VRAR_API int vrar_all_gather(const void* const rank_in[], void* const rank_out[]
  */
 VRAR_API int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype);
 
+/*
+ * Base name of the kernel that vrar_allreduce(.., P, n, dtype, algo, ..) would
+ * launch under the current settings (AUTO resolved as vrar_allreduce resolves
+ * it, the payload wire, the VRAR_WRITE_KERNEL override), e.g.
+ * "k_twostage_write_async". Write mode has three kernels with one result:
+ * "k_twostage_write" (plain), "k_twostage_write_staged" (bulk copies into
+ * shared memory by one producer lane), "k_twostage_write_async" (per-thread
+ * async copies into shared memory), chosen per shape from the same measured
+ * table as vrar_select_algo. For profilers and benchmarks; the sources have
+ * no counterpart. Returns a static string, or NULL for invalid arguments
+ * (P outside 1..VRAR_MAX_RANKS, unknown dtype or algorithm). Launches nothing.
+ */
+VRAR_API const char* vrar_kernel_name(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t algo);
+
 /* Group size L used by VRAR_ALGO_HIER (default 8). Returns VRAR_OK or
  * VRAR_EINVAL (L < 1 or L > VRAR_MAX_RANKS). Process-wide setting. */
 VRAR_API int vrar_set_group_size(int L);

@@ -149,12 +149,37 @@ def test_selector_table_entries():
     assert vrar.select_algo(1, 1 << 20, bf) == "oneshot"            # a copy
     assert vrar.select_algo(2, 1 << 20, bf) == "oneshot"            # 2 MiB at 2 ranks
     assert vrar.select_algo(2, 4 << 20, bf) == "twostage_write"     # 8 MiB at 2 ranks
-    assert vrar.select_algo(8, 65536, bf) == "oneshot"              # 128 KiB at 8 ranks
     assert vrar.select_algo(8, 524288, bf) == "twostage_write"      # 1 MiB at 8 ranks (the decode shape)
     assert vrar.select_algo(8, 117440512, bf) == "twostage_write"   # prefill
     assert vrar.select_algo(32, 16384, bf) == "twostage_write"      # 32 KiB at 32 ranks
-    assert vrar.select_algo(8, 65536, torch.float32) == "oneshot"   # 256 KiB in fp32
     assert vrar.select_algo(8, 524288, torch.float16) == "twostage_write"
+
+
+def test_kernel_name():
+    """Which kernel a call launches: write mode has three kernels with one result."""
+    bf = torch.bfloat16
+    if os.environ.get("VRAR_WRITE_KERNEL") or os.environ.get("VRAR_ALGO"):
+        pytest.skip("an override is set in the environment")
+    assert vrar.kernel_name(8, 524288, bf, "oneshot") == "k_oneshot"
+    assert vrar.kernel_name(8, 524288, bf, "twostage") == "k_twostage"
+    assert vrar.kernel_name(8, 524288, bf, "rd") == "k_rd"
+    assert vrar.kernel_name(32, 524288, bf, "hier") == "k_hier"
+    assert vrar.kernel_name(8, 524288, bf, "auto") == "k_twostage_write_async"       # the decode shape
+    assert vrar.kernel_name(8, 117440512, bf, "auto") == "k_twostage_write_staged"   # prefill
+    assert vrar.kernel_name(1, 1000, bf, "auto") == "k_oneshot"
+    for P in (1, 2, 3, 8, 13, 32):
+        for n in (0, 1, 65536, 524288, 1 << 24):
+            for dt in (bf, torch.float16, torch.float32):
+                assert vrar.kernel_name(P, n, dt, "twostage_write").startswith("k_twostage_write")
+    vrar.set_payload_wire("fp32")
+    try:
+        assert vrar.kernel_name(8, 524288, bf, "rd") == "k_rd_wide"
+        assert vrar.kernel_name(8, 524288, torch.float32, "rd") == "k_rd"   # fp32 data already travels as fp32
+    finally:
+        vrar.set_payload_wire("element")
+    for bad in ((0, 10), (33, 10)):
+        with pytest.raises(vrar.VrarError):
+            vrar.kernel_name(bad[0], bad[1], bf, "auto")
 
 
 def test_payload_wire_setting():

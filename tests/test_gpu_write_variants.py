@@ -1,9 +1,11 @@
-"""Both write-mode kernels (plain and shared-memory staged) against the oracle.
+"""The three write-mode kernels (plain, bulk-copy staged, per-thread async
+copies) against the oracle.
 
-The per-shape table sends each shape to one of the two kernels, so this test
+The per-shape table sends each shape to one of the kernels, so this test
 forces each in turn (VRAR_WRITE_KERNEL is read once per process, hence the
-child processes) over shapes with ragged tails, up to 32 ranks, both dtypes,
-with and without the start/end barriers.
+child processes) over shapes with ragged tails, up to 32 ranks, all three
+dtypes, with and without the start/end barriers, and with a CTA budget (which
+changes the grid and, for the staged and async kernels, the stage depth).
 """
 
 import os
@@ -26,21 +28,25 @@ CHILD = textwrap.dedent("""
     import oracle, synth
     from util import from_np, gen, to_np, bits_of
     for dtype in ("bf16", "fp32", "fp16"):
-        for P, n in ((1, 1001), (2, 7), (3, 66_001), (8, 9), (8, 300_007), (16, 70_001), (32, 33_333), (32, 1_000_003)):
+        for P, n in ((1, 1001), (2, 7), (3, 66_001), (8, 9), (8, 300_007), (13, 4_099), (16, 70_001), (24, 50_021),
+                     (32, 33_333), (32, 1_000_003)):
             xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P + n)
             want = oracle.allreduce("twostage_write", xs, dtype)
-            for edge in (False, True):
+            for edge, cap in ((False, 0), (True, 0), (False, 64)):
                 vrar.set_edge_sync(edge)
+                vrar.set_max_ctas(cap)
                 outs = vrar.all_reduce([from_np(x, dtype).cuda() for x in xs], algo="twostage_write")
                 rc, info = vrar.query_status()
                 assert rc == 0, (rc, info)
                 for p in range(P):
-                    assert np.array_equal(bits_of(to_np(outs[p])), bits_of(want[p])), (dtype, P, n, edge, p)
+                    assert np.array_equal(bits_of(to_np(outs[p])), bits_of(want[p])), (dtype, P, n, edge, cap, p)
+            vrar.set_edge_sync(False)
+            vrar.set_max_ctas(0)
     print("ok")
 """)
 
 
-@pytest.mark.parametrize("variant", ["plain", "staged"])
+@pytest.mark.parametrize("variant", ["plain", "staged", "async"])
 def test_write_kernel_variant_matches_oracle(variant):
     env = dict(os.environ, VRAR_WRITE_KERNEL=variant)
     code = CHILD.format(root=ROOT, tests=os.path.join(ROOT, "tests"))
