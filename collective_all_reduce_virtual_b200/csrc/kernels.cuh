@@ -26,22 +26,23 @@ __device__ __forceinline__ int64_t lo_of(int64_t part, int64_t piece, int64_t to
 // One-shot [CAR, the 1-stage kernel]: every rank reads all P inputs and
 // reduces the whole vector into its own output, between start and end
 // barriers. The P CTAs with the same b read the same items at about the same
-// time, so all but the first read of each line hit L2.
-template <class D>
-__global__ void __launch_bounds__(kThreads, 2) k_oneshot(const KArgs a) {
+// time, so all but the first read of each line hit L2. T threads per CTA:
+// small messages run faster as more, smaller CTAs.
+template <class D, int T = kThreads>
+__global__ void __launch_bounds__(T, 2) k_oneshot(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
   // Rank r's CTAs prefetch input r only: all P ranks read the same items.
   if (threadIdx.x == 0)
-    prefetch_items<D>(a.ptr.in[c.r], static_cast<int64_t>(c.b) * kThreads, kThreads, a.n);
+    prefetch_items<D>(a.ptr.in[c.r], static_cast<int64_t>(c.b) * T, T, a.n);
   pdl_wait();
   if (a.edge_sync) {
     cta_publish_flag(c, cta_take_ticket(a));
     if (!block_barrier(a, c, kPhStart)) return;
   }
-  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
+  const int64_t stride = static_cast<int64_t>(a.B) * T;
   void* out = a.ptr.out[c.r];
-  for (int64_t it = static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < a.items; it += stride)
+  for (int64_t it = static_cast<int64_t>(c.b) * T + threadIdx.x; it < a.items; it += stride)
     store_item<D, true>(out, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
   if (a.edge_sync) block_barrier(a, c, kPhEnd);
 }
@@ -281,7 +282,11 @@ __global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(cons
 // threads issue copies in parallel (the staged kernel's single producer lane
 // issues P bulk copies per tile one after another, which is what limits it
 // on small messages at many ranks). Shared memory: S * P * TI * 16 bytes.
-template <class D, int TI, int S>
+//
+// With kScatter the same kernel is the standalone reduce-scatter: rank r's
+// slice is its chunk (n / P elements, a whole number of items) and the result
+// goes to out[r] only, at the chunk's local offset.
+template <class D, int TI, int S, bool kScatter = false>
 __global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   pdl_trigger();
@@ -329,14 +334,18 @@ __global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
       acc.init(ld_shared_v4(src));
       for (int p = 1; p < a.P; ++p) acc.add(ld_shared_v4(src + p * (TI * 16)));
       const uint4 v = acc.round();
-      for (int j = 0; j < a.P; ++j) {
-        const int q = (c.r + j) % a.P;
-        st_stream(static_cast<typename D::E*>(a.ptr.out[q]) + it * D::VE, v);
+      if (kScatter) {
+        st_stream(static_cast<typename D::E*>(a.ptr.out[c.r]) + (it - lo) * D::VE, v);
+      } else {
+        for (int j = 0; j < a.P; ++j) {
+          const int q = (c.r + j) % a.P;
+          st_stream(static_cast<typename D::E*>(a.ptr.out[q]) + it * D::VE, v);
+        }
       }
     }
   }
   cp_async_wait<0>();
-  if (threadIdx.x == 0 && c.b == 0 && full_items < a.items && full_items >= lo && full_items < hi) {
+  if (!kScatter && threadIdx.x == 0 && c.b == 0 && full_items < a.items && full_items >= lo && full_items < hi) {
     const uint4 v = reduce_item<D>(a.ptr, 0, a.P, full_items, a.n);
     for (int p = 0; p < a.P; ++p) store_item<D, true>(a.ptr.out[p], full_items, a.n, v);
   }
@@ -633,7 +642,9 @@ __global__ void __launch_bounds__(kThreads) k_hier_wide(const KArgs a) {
 // Standalone reduce-scatter [NVRAR phase 1 over one group]: rank p writes
 // elements [p*m, (p+1)*m) of the ascending-rank sum into out[p], m = n / P.
 // Needs no flags. 16-byte path when m is a multiple of the item size (so
-// every slice starts on a 16-byte boundary), element path otherwise.
+// every slice starts on a 16-byte boundary), element path otherwise. Up to
+// 1 MiB per rank the async-copy write kernel in its scatter form is used
+// instead of the 16-byte path here.
 template <class D>
 __global__ void __launch_bounds__(kThreads, 2) k_reduce_scatter(const KArgs a) {
   pdl_trigger();
@@ -663,31 +674,33 @@ __global__ void __launch_bounds__(kThreads, 2) k_reduce_scatter(const KArgs a) {
 }
 
 // Standalone all-gather [NVRAR phase 3 over one group], push form: rank s
-// reads its n/P elements once and streams them to offset s*m of all P outputs.
+// reads its n/P elements and streams them to offset s*m of all P outputs.
+// The P destinations are split over G = a.chunks groups of CTAs (group g
+// writes outputs g, g+G, g+2G, ...), so that a short slice still spreads over
+// many SMs; each group reads the slice once more, from L2.
 template <class D>
 __global__ void __launch_bounds__(kThreads, 2) k_all_gather(const KArgs a) {
   pdl_trigger();
-  const int s = static_cast<int>(blockIdx.x % a.P), b = static_cast<int>(blockIdx.x / a.P);
+  const int s = static_cast<int>(blockIdx.x % a.P);
+  const int rest = static_cast<int>(blockIdx.x / a.P);
+  const int b = rest % a.B, g = rest / a.B, G = a.chunks;
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
   const int64_t t0 = static_cast<int64_t>(b) * kThreads + threadIdx.x;
   const int64_t m = a.n / a.P;
-  if (m % D::VE == 0 && threadIdx.x == 0)
+  if (m % D::VE == 0 && threadIdx.x == 0 && g == 0)
     prefetch_items<D>(a.ptr.in[s], static_cast<int64_t>(b) * kThreads, kThreads, m);
   pdl_wait();
   if (m % D::VE == 0) {
     const int64_t mi = m / D::VE;
     for (int64_t j = t0; j < mi; j += stride) {
       const uint4 v = load_item_input<D>(a.ptr.in[s], j, m);
-      for (int jj = 0; jj < a.P; ++jj) {
-        const int p = (s + jj) % a.P;
-        store_item<D, true>(a.ptr.out[p], s * mi + j, a.n, v);
-      }
+      for (int q = g; q < a.P; q += G) store_item<D, true>(a.ptr.out[q], s * mi + j, a.n, v);
     }
   } else {
     using E = typename D::E;
     for (int64_t e = t0; e < m; e += stride) {
       const E v = static_cast<const E*>(a.ptr.in[s])[e];
-      for (int p = 0; p < a.P; ++p) static_cast<E*>(a.ptr.out[p])[s * m + e] = v;
+      for (int q = g; q < a.P; q += G) static_cast<E*>(a.ptr.out[q])[s * m + e] = v;
     }
   }
 }

@@ -351,6 +351,19 @@ def test_reduce_scatter_and_all_gather(dtype):
             sl = gen(P, m, dtype, synth.normal(0.0, 1.0), seed=P * m)
             got = [to_np(o) for o in vrar.all_gather(_dev(sl, dtype))]
             assert_bits(got, oracle.all_gather(sl, dtype), f"AG P={P} m={m}")
+    # Many tiles per CTA, with and without a CTA budget (which deepens the
+    # stages): 32,768 elements per chunk take the async-copy form (at most
+    # 1 MiB per rank), 131,072 the 16-byte plain kernel.
+    for P, m in ((8, 32_768), (8, 131_072)):
+        xs = gen(P, m * P, dtype, synth.normal(0.0, 1.0), seed=7)
+        want = oracle.reduce_scatter(xs, dtype)
+        for cap in (0, 16):
+            vrar.set_max_ctas(cap)
+            try:
+                got = [to_np(o) for o in vrar.reduce_scatter(_dev(xs, dtype))]
+            finally:
+                vrar.set_max_ctas(0)
+            assert_bits(got, want, f"RS P={P} m={m} max_ctas={cap}")
     rc, info = vrar.query_status()
     assert rc == 0, info
 
