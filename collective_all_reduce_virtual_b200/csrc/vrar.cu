@@ -348,8 +348,8 @@ int write_kernel_override() {
 // 'A' write mode with the per-thread async-copy kernel, 'S' write mode with
 // the bulk-copy staged kernel, 'P' write mode with the plain kernel. Rows:
 // P <= 2, 4, 8, 16, 32; columns: bytes per rank <= 32 KiB, 64 KiB, ...,
-// 8 MiB, and above. One-shot keeps small messages at two ranks (one pass,
-// its re-reads served by L2). The async write kernel wins almost everywhere
+// 8 MiB, and above. One-shot keeps small messages at two and four ranks (one
+// pass, its re-reads served by L2). The async write kernel wins almost everywhere
 // else: every thread keeps all P loads of its items in flight, with no
 // serial issue. From 8 MiB per rank at 4-16 ranks the bulk-copy pipeline
 // streams a little better, and at 32 ranks from 4 MiB the plain kernel
@@ -357,7 +357,7 @@ int write_kernel_override() {
 // percent.
 constexpr char kChoice[5][10] = {
     {'O', 'O', 'O', 'O', 'O', 'O', 'O', 'A', 'A', 'A'},  // P <= 2
-    {'A', 'A', 'A', 'O', 'O', 'A', 'A', 'A', 'S', 'A'},  // P <= 4
+    {'O', 'O', 'A', 'O', 'O', 'A', 'A', 'A', 'S', 'A'},  // P <= 4
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 8
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 16
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'P'},  // P <= 32
