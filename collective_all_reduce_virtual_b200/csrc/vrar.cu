@@ -545,6 +545,11 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
 
   int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
   const bool wide = wide_wire(algo, dtype);
+  // HIER keeps at most two payload pieces per thread: its in-group phases
+  // already keep L loads and L stores per piece in flight, and more pieces
+  // cost registers (measured, 4 groups x 8: 50 vs 56 us at 2 MiB per rank,
+  // 226 vs 251 us at 8 MiB, two pieces against four).
+  if (algo == VRAR_ALGO_HIER && !wide) C = std::min(C, 2);
   if (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER) {
     const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
     const int64_t work = algo == VRAR_ALGO_RD ? items : (items + L - 1) / L;
