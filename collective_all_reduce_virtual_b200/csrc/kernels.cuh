@@ -489,9 +489,11 @@ __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
 // ascending order, one rounding. Phase 2 (inter-group recursive doubling):
 // log2 G steps of fused-payload exchange with partner (g XOR 2^s, l). Phase 3
 // (in-group all-gather): rank (g, l) streams slice l into the outputs of all
-// L ranks of group g. Slices are cut into C chunks as in k_rd.
-template <class D, int C>
-__global__ void __launch_bounds__(kThreads) k_hier(const KArgs a) {
+// L ranks of group g. Slices are cut into C chunks as in k_rd. kMinBlocks 2
+// limits registers to fit two CTAs per SM (more threads in flight when a call
+// needs several rounds over its items).
+template <class D, int C, int kMinBlocks = 1>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) k_hier(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
   const int L = a.L, g = c.r / L, l = c.r % L;

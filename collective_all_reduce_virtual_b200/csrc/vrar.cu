@@ -414,6 +414,24 @@ KernelFn oneshot_small_dt(vrar_dtype_t dt) {
                            : k_oneshot<F32T, kSmallThreads>;
 }
 
+// HIER (element wire) by size, measured at 4 groups x 8 ranks: up to 256 KiB
+// per rank one 512-thread CTA per SM (7.8 us; the call is one round over its
+// items and the 64-register build spills); above it two CTAs per SM, with one
+// payload piece per thread up to 2 MiB per rank (43 vs 50 us at 2 MiB) and
+// two above (204 vs 226 us at 8 MiB).
+constexpr size_t kHierOneCtaBytes = 256 << 10;
+constexpr size_t kHierOnePieceBytes = 2 << 20;
+
+template <class D>
+KernelFn hier_two_per_sm(int C) {
+  return C <= 1 ? k_hier<D, 1, 2> : k_hier<D, 2, 2>;
+}
+
+KernelFn hier_two_per_sm_dt(vrar_dtype_t dt, int C) {
+  return dt == VRAR_BF16 ? hier_two_per_sm<Bf16T>(C) : dt == VRAR_FP16 ? hier_two_per_sm<F16T>(C)
+                                                                      : hier_two_per_sm<F32T>(C);
+}
+
 template <class D>
 KernelFn async_rs_kernel(int S) {
   switch (S) {
@@ -548,7 +566,8 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   // HIER keeps at most two payload pieces per thread: its in-group phases
   // already keep L loads and L stores per piece in flight, and more pieces
   // cost registers (measured, 4 groups x 8: 50 vs 56 us at 2 MiB per rank,
-  // 226 vs 251 us at 8 MiB, two pieces against four).
+  // 226 vs 251 us at 8 MiB, two pieces against four). Above 256 KiB per rank
+  // it also runs two CTAs per SM (below).
   if (algo == VRAR_ALGO_HIER && !wide) C = std::min(C, 2);
   if (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER) {
     const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
@@ -557,6 +576,10 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
              : rd_chunks_for_dt(dtype, algo, C, work, P, dev, ws->sms);
   }
   KernelFn fn = wide ? pick_wide_dt(dtype, algo, C) : pick_kernel_dt(dtype, algo, C);
+  if (algo == VRAR_ALGO_HIER && !wide && n * elem_size(dtype) > kHierOneCtaBytes) {
+    if (n * elem_size(dtype) <= kHierOnePieceBytes) C = 1;
+    fn = hier_two_per_sm_dt(dtype, C);
+  }
   if (!fn) return VRAR_EINVAL;
 
   KArgs a;
