@@ -437,18 +437,23 @@ def test_spin_stats_count_timeouts():
 
 # ---- failure detection: bounded waits, no GPU fault ----------------------------------------------
 
-@pytest.mark.parametrize("algo,P,L,edge,phase", [
-    ("rd_fp32wire", 4, 8, True, 4),
-    ("oneshot", 4, 8, True, 1),
-    ("twostage", 4, 8, False, 2),
-    ("twostage_write", 8, 8, True, 1),
-    ("rd", 4, 8, True, 4),
-    ("hier", 8, 2, True, 4),
+@pytest.mark.parametrize("algo,P,L,edge,phase,n", [
+    ("rd_fp32wire", 4, 8, True, 4, 40_000),
+    ("oneshot", 4, 8, True, 1, 40_000),
+    ("twostage", 4, 8, False, 2, 40_000),
+    ("twostage_write", 8, 8, True, 1, 40_000),      # async-copy write kernel
+    ("twostage_write", 8, 8, True, 1, 4_194_304),   # 8 MiB per rank: bulk-copy staged kernel
+    ("rd", 4, 8, True, 4, 40_000),
+    ("hier", 8, 2, True, 4, 40_000),
+    ("hier", 8, 2, True, 4, 600_000),               # above 256 KiB per rank: two CTAs per SM
 ])
-def test_missing_rank_times_out_and_recovers(algo, P, L, edge, phase):
+def test_missing_rank_times_out_and_recovers(algo, P, L, edge, phase, n):
     """A rank that never posts (fault mask) makes its peers' waits run out; the
     kernel records VRAR_ETIMEDOUT and exits, and the next call works."""
-    xs = gen(P, 40_000, "bf16", synth.normal(0.0, 1.0), seed=5)
+    xs = gen(P, n, "bf16", synth.normal(0.0, 1.0), seed=5)
+    if algo == "twostage_write":  # the case must reach the kernel it is there for
+        want_kernel = {40_000: "k_twostage_write_async", 4_194_304: "k_twostage_write_staged"}[n]
+        assert vrar.kernel_name(P, n, torch.bfloat16, algo) == want_kernel
     d_in = _dev(xs, "bf16")
     vrar.set_group_size(L)
     vrar.set_edge_sync(edge)
