@@ -101,6 +101,29 @@ def b_min_bytes(P: int, n: int, esz: int) -> int:
     return 2 * P * n * esz
 
 
+def b_alg_bytes(algo: str, P: int, n: int, esz: int, L: int = 8, fp32_wire: bool = False) -> int:
+    """Bytes an algorithm's own loads and stores ask for (each input and output
+    counted at every access; repeat reads may hit L2). One-shot: every rank
+    reads all P inputs, (P^2 + P) n s. Two-stage pull: (3P - 1) n s. Write mode:
+    2 P n s. Recursive doubling: inputs and outputs plus, per step, every rank's
+    payload words written and read, 2 n s each way ({32 data bits | 32-bit
+    sequence} per 8 bytes; fp32 partials of 16-bit data double that). HIER:
+    2 P n s plus the same payload traffic on 1/L of the data over log2(P/L)
+    steps."""
+    wire = 2 if (fp32_wire and esz == 2) else 1
+    if algo == "oneshot":
+        return (P * P + P) * n * esz
+    if algo == "twostage":
+        return (3 * P - 1) * n * esz
+    if algo == "twostage_write":
+        return 2 * P * n * esz
+    if algo == "rd":
+        return P * n * esz * (2 + 4 * wire * int(math.log2(P)))
+    if algo == "hier":
+        return int((2 * P + 4 * wire * math.log2(P // L) * P / L) * n * esz)
+    raise ValueError(algo)
+
+
 def rotation_sets(set_bytes: int, l2_bytes: int = L2_BYTES, cap: int = 64) -> int:
     """Buffer sets to rotate through so that the total exceeds 3x the L2 size."""
     return max(1, min(cap, math.ceil(3 * l2_bytes / max(1, set_bytes))))
@@ -362,11 +385,16 @@ def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1
     return ms / steps
 
 
-def entry(wl: Workload, t_s: float, peak: float):
+def entry(wl: Workload, t_s: float, peak: float, algo: str):
+    """One timing: busbw, and the fraction of the measured HBM bandwidth on
+    B_min (algorithm-independent) and on B_alg (the algorithm's own traffic)."""
     bw = busbw_gbs(wl.P, wl.n, wl.esz, t_s)
     ach = b_min_bytes(wl.P, wl.n, wl.esz) / t_s / 1e9
+    if algo == "auto":
+        algo = wl.vrar.select_algo(wl.P, wl.n, TDT[wl.dt])
+    b_alg = b_alg_bytes(algo, wl.P, wl.n, wl.esz, wl.spec.get("L", 8), wl.spec.get("wire") == "fp32")
     return {"us": round(t_s * 1e6, 3), "busbw_gbs": round(bw, 1), "hbm_gbs_bmin": round(ach, 1),
-            "frac_bmin": round(ach / peak, 4)}
+            "frac_bmin": round(ach / peak, 4), "frac_alg": round(b_alg / t_s / 1e9 / peak, 4)}
 
 
 def measure_e2e(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None):
@@ -485,7 +513,7 @@ def run_vrar(args):
     per_algo = {}
     if not args.quick:
         for algo in ("oneshot", "twostage", "twostage_write", "rd"):
-            per_algo[algo] = entry(wl, measure_algo(wl, algo, 200, 5, world, device) / 1e3, peak)
+            per_algo[algo] = entry(wl, measure_algo(wl, algo, 200, 5, world, device) / 1e3, peak, algo)
     wl.free()
 
     # Warm L2: the same buffers every call (inputs and outputs, 16 MiB, stay in
@@ -494,7 +522,7 @@ def run_vrar(args):
     if not args.quick:
         ww = Workload(WORKLOAD, device, rotate=False)
         for algo in ("auto", "oneshot", "twostage", "twostage_write", "rd"):
-            warm[algo] = entry(ww, measure_algo(ww, algo, 200, 5, world, device) / 1e3, peak)
+            warm[algo] = entry(ww, measure_algo(ww, algo, 200, 5, world, device) / 1e3, peak, algo)
         ww.free()
 
     sweep = []
@@ -509,7 +537,7 @@ def run_vrar(args):
                    "kernel": vrar.kernel_name(w.P, w.n, TDT[w.dt], "auto")}
             for algo in spec["algos"]:
                 k = spec.get("steps", 200)
-                row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device) / 1e3, peak)
+                row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device) / 1e3, peak, algo)
             for kind in spec.get("collectives", ()):
                 # RS moves P*n*s in and n*s out; AG n*s in and P*n*s out: (P+1)*n*s either way.
                 t = measure_collective(w, kind, spec.get("steps", 200), 3, world, device) / 1e3

@@ -19,6 +19,28 @@ def test_busbw_and_bytes():
     assert bench.b_min_bytes(8, 524288, 2) == 16 * 1024 * 1024
 
 
+def test_algorithmic_bytes_per_algorithm():
+    """B_alg counted access by access for small cases, against the closed forms."""
+    s = 2
+    # write mode moves exactly the minimum: P inputs read, P outputs written
+    assert bench.b_alg_bytes("twostage_write", 8, 1, s) == bench.b_min_bytes(8, 1, s) == 32
+    # one-shot: every one of P ranks reads P inputs and writes its output
+    assert bench.b_alg_bytes("oneshot", 8, 1, s) == (8 * 8 + 8) * s
+    # pull two-stage: P n s of inputs read, n s of reduced chunks written, then every rank reads
+    # and writes the (P - 1) chunks it lacks: P + 1 + 2 (P - 1) = 3P - 1 times n s
+    assert bench.b_alg_bytes("twostage", 8, 1, s) == (3 * 8 - 1) * s
+    # recursive doubling, 8 ranks: inputs + outputs, and per step each rank writes and reads
+    # 8 bytes of payload per 4 data bytes
+    steps, per_step = 3, 2 * (8 * 1 * s * 2)
+    assert bench.b_alg_bytes("rd", 8, 1, s) == 2 * 8 * 1 * s + steps * per_step
+    assert bench.b_alg_bytes("rd", 8, 1, s, fp32_wire=True) == 2 * 8 * 1 * s + steps * 2 * per_step
+    assert bench.b_alg_bytes("rd", 8, 1, 4, fp32_wire=True) == bench.b_alg_bytes("rd", 8, 1, 4)
+    # hierarchical 4 x 8: 2 P n s plus 2 steps of payload on n / 8 per rank: 3 P n s
+    assert bench.b_alg_bytes("hier", 32, 8, s, L=8) == 3 * 32 * 8 * s
+    with pytest.raises(ValueError):
+        bench.b_alg_bytes("auto", 8, 1, s)
+
+
 def test_rotation_exceeds_l2():
     for set_bytes in (2 << 20, 16 << 20, 128 << 20, 3758096384):
         R = bench.rotation_sets(set_bytes)
