@@ -401,10 +401,11 @@ int async_stages(int P, size_t bytes_per_rank, bool deep) {
   return s >= 8 ? 8 : s >= 6 ? 6 : s >= 4 ? 4 : 3;
 }
 
-// One-shot on small messages (at most 256 KiB per rank): 128-thread CTAs,
-// more of them, measured faster there (1.34 vs 1.55 us at 2 ranks x 128 KiB);
-// from 512 KiB per rank the 512-thread CTAs are faster.
-constexpr size_t kOneshotSmallBytes = 256 << 10;
+// One-shot on small messages (at most 1 MiB of input over all P ranks):
+// 128-thread CTAs, more of them, measured faster there (1.46 vs 1.60 us at
+// 2 ranks x 128 KiB, 2.37 vs 2.64 us at 8 x 128 KiB); above it the 512-thread
+// CTAs are faster (2.62 vs 3.59 us at 8 x 256 KiB, 4.06 vs 5.86 at 16 x 128 KiB).
+constexpr size_t kOneshotSmallBytes = 1 << 20;
 constexpr size_t kRsAsyncMaxBytes = 1 << 20;  // reduce-scatter: async scatter form up to here (bytes per rank)
 constexpr int kSmallThreads = 128;
 
@@ -651,7 +652,7 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     return launch(sf, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), 32 + ti, smem);
   }
   int threads = kThreads;
-  if (algo == VRAR_ALGO_ONESHOT && n * elem_size(dtype) <= kOneshotSmallBytes) {
+  if (algo == VRAR_ALGO_ONESHOT && static_cast<size_t>(P) * n * elem_size(dtype) <= kOneshotSmallBytes) {
     fn = oneshot_small_dt(dtype);
     threads = kSmallThreads;
   }
