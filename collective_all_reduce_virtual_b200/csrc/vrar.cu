@@ -416,10 +416,10 @@ KernelFn oneshot_small_dt(vrar_dtype_t dt) {
 }
 
 // HIER (element wire) by size, measured at 4 groups x 8 ranks: up to 256 KiB
-// per rank one 512-thread CTA per SM (7.8 us; the call is one round over its
-// items and the 64-register build spills); above it two CTAs per SM, with one
-// payload piece per thread up to 2 MiB per rank (43 vs 50 us at 2 MiB) and
-// two above (204 vs 226 us at 8 MiB).
+// per rank one 512-thread CTA per SM (7.8 vs 9.9 us; the call is one round
+// over its items and the 64-register build spills); above it two CTAs per SM
+// (43 vs 50 us at 2 MiB with one piece per thread, 204 vs 226 us at 8 MiB
+// with two).
 constexpr size_t kHierOneCtaBytes = 256 << 10;
 constexpr size_t kHierOnePieceBytes = 2 << 20;
 
@@ -564,12 +564,13 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
 
   int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
   const bool wide = wide_wire(algo, dtype);
-  // HIER keeps at most two payload pieces per thread: its in-group phases
-  // already keep L loads and L stores per piece in flight, and more pieces
-  // cost registers (measured, 4 groups x 8: 50 vs 56 us at 2 MiB per rank,
-  // 226 vs 251 us at 8 MiB, two pieces against four). Above 256 KiB per rank
-  // it also runs two CTAs per SM (below).
-  if (algo == VRAR_ALGO_HIER && !wide) C = std::min(C, 2);
+  // HIER keeps one payload piece per thread up to 2 MiB per rank and at most
+  // two above: its in-group phases already keep L loads and L stores per
+  // piece in flight, and more pieces cost registers (measured, 4 groups x 8,
+  // both wires; e.g. 226 vs 251 us at 8 MiB, two pieces against four, and
+  // 78 vs 84 us at 2 MiB with fp32 partials, one against two). Above 256 KiB
+  // per rank the element-wire kernel also runs two CTAs per SM (below).
+  if (algo == VRAR_ALGO_HIER) C = n * elem_size(dtype) <= kHierOnePieceBytes ? 1 : std::min(C, 2);
   if (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER) {
     const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
     const int64_t work = algo == VRAR_ALGO_RD ? items : (items + L - 1) / L;
@@ -577,10 +578,7 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
              : rd_chunks_for_dt(dtype, algo, C, work, P, dev, ws->sms);
   }
   KernelFn fn = wide ? pick_wide_dt(dtype, algo, C) : pick_kernel_dt(dtype, algo, C);
-  if (algo == VRAR_ALGO_HIER && !wide && n * elem_size(dtype) > kHierOneCtaBytes) {
-    if (n * elem_size(dtype) <= kHierOnePieceBytes) C = 1;
-    fn = hier_two_per_sm_dt(dtype, C);
-  }
+  if (algo == VRAR_ALGO_HIER && !wide && n * elem_size(dtype) > kHierOneCtaBytes) fn = hier_two_per_sm_dt(dtype, C);
   if (!fn) return VRAR_EINVAL;
 
   KArgs a;
