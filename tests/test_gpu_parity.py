@@ -97,8 +97,11 @@ def test_integer_inputs_give_exact_sums(dtype):
         exact = np.stack([oracle.to_float(x, dtype) for x in xs]).astype(np.int64).sum(axis=0)
         for algo, L in algos_for(P):
             got = run(algo, xs, dtype, L=L)
-            for g in got:
+            for p, g in enumerate(got):
                 assert (oracle.to_float(g, dtype) == exact).all(), f"{algo} L={L} P={P}"
+                # A real reduction happened: a rank's output is not its own input
+                # (a one-rank "collective" that copies would pass a same-value check).
+                assert (bits_of(g) != bits_of(xs[p])).mean() > 0.5, f"{algo} L={L} P={P} rank {p} copied its input"
 
 
 def test_golden_order_cases_on_gpu():
