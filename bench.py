@@ -385,6 +385,19 @@ def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1
     return ms / steps
 
 
+class nvtx:
+    """An NVTX range around a phase of the benchmark (visible in profilers)."""
+
+    def __init__(self, name: str):
+        self.name = name
+
+    def __enter__(self):
+        torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        torch.cuda.nvtx.range_pop()
+
+
 def entry(wl: Workload, t_s: float, peak: float, algo: str):
     """One timing: busbw, and the fraction of the measured HBM bandwidth on
     B_min (algorithm-independent) and on B_alg (the algorithm's own traffic)."""
@@ -393,8 +406,9 @@ def entry(wl: Workload, t_s: float, peak: float, algo: str):
     if algo == "auto":
         algo = wl.vrar.select_algo(wl.P, wl.n, TDT[wl.dt])
     b_alg = b_alg_bytes(algo, wl.P, wl.n, wl.esz, wl.spec.get("L", 8), wl.spec.get("wire") == "fp32")
-    return {"us": round(t_s * 1e6, 3), "busbw_gbs": round(bw, 1), "hbm_gbs_bmin": round(ach, 1),
-            "frac_bmin": round(ach / peak, 4), "frac_alg": round(b_alg / t_s / 1e9 / peak, 4)}
+    return {"us": round(t_s * 1e6, 3), "algbw_gbs": round(wl.n * wl.esz / t_s / 1e9, 1), "busbw_gbs": round(bw, 1),
+            "hbm_gbs_bmin": round(ach, 1), "frac_bmin": round(ach / peak, 4),
+            "frac_alg": round(b_alg / t_s / 1e9 / peak, 4)}
 
 
 def measure_e2e(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None):
@@ -504,11 +518,13 @@ def run_vrar(args):
     algo_auto = vrar.select_algo(wl.P, wl.n, TDT[wl.dt])
 
     # The timed steps: exactly K AUTO calls.
-    t_step_ms = measure_algo(wl, "auto", args.steps, args.warmup, world, device)
+    with nvtx("timed steps"):
+        t_step_ms = measure_algo(wl, "auto", args.steps, args.warmup, world, device)
     t_s = t_step_ms / 1e3
 
     # e2e through the public call with host buffers.
-    e2e_ms, h2d, d2h = measure_e2e(wl, "auto", max(3, min(args.steps, 50)), args.warmup, world, device)
+    with nvtx("e2e"):
+        e2e_ms, h2d, d2h = measure_e2e(wl, "auto", max(3, min(args.steps, 50)), args.warmup, world, device)
 
     per_algo = {}
     if not args.quick:
