@@ -207,7 +207,10 @@ VRAR_API int vrar_get_edge_sync(void);
  * budget leaves SMs to work running concurrently on other streams, e.g. the
  * partner micro-batch's GEMMs while this all-reduce runs on a communication
  * stream; the all-reduce is bound by memory bandwidth, which a fraction of
- * the SMs can already draw. Process-wide setting. */
+ * the SMs can already draw. With a budget of at most one CTA per SM the
+ * write-mode and reduce-scatter kernels keep more bytes in flight per CTA
+ * (deeper shared-memory stages). Results do not depend on the budget.
+ * Process-wide setting. */
 VRAR_API int vrar_set_max_ctas(int n);
 VRAR_API int vrar_get_max_ctas(void);
 
@@ -221,7 +224,8 @@ VRAR_API uint64_t vrar_get_spin_timeout_ns(void);
  * current device: VRAR_OK, or VRAR_ETIMEDOUT if any wait of any call since
  * the last query ran out of time. If info is not NULL it receives details of
  * the first failure: info[0] = call sequence number, info[1] = phase
- * (1 start, 2 mid, 3 end, 4 payload), info[2] = waiting rank, info[3] = block.
+ * (1 start, 2 mid, 3 end, 4 payload, 5 shared-memory stage of the bulk-copy
+ * write kernel), info[2] = waiting rank, info[3] = block.
  */
 VRAR_API int vrar_query_status(vrar_stream_t stream, uint32_t info[4]);
 
