@@ -49,15 +49,16 @@ __global__ void __launch_bounds__(T, 2) k_oneshot(const KArgs a) {
 
 // 2-stage [CAR "cross_device_reduce_2stage"], pull mode. Stage 1: rank r
 // reduces slice r (ceil(items / P) items) over all P inputs into out[r]. Mid
-// barrier. Stage 2: rank r copies every other slice s out of out[s].
-template <class D>
-__global__ void __launch_bounds__(kThreads) k_twostage(const KArgs a) {
+// barrier. Stage 2: rank r copies every other slice s out of out[s]. T threads
+// per CTA (the library launches 256: more, smaller CTAs per column barrier).
+template <class D, int T = kThreads>
+__global__ void __launch_bounds__(T) k_twostage(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
   {
     const int64_t piece = (a.items + a.P - 1) / a.P;
-    const int64_t first = lo_of(c.r, piece, a.items) + static_cast<int64_t>(c.b) * kThreads;
-    const int64_t count = min(static_cast<int64_t>(kThreads), lo_of(c.r + 1, piece, a.items) - first);
+    const int64_t first = lo_of(c.r, piece, a.items) + static_cast<int64_t>(c.b) * T;
+    const int64_t count = min(static_cast<int64_t>(T), lo_of(c.r + 1, piece, a.items) - first);
     if (threadIdx.x < a.P) prefetch_items<D>(a.ptr.in[threadIdx.x], first, count, a.n);
   }
   pdl_wait();
@@ -66,8 +67,8 @@ __global__ void __launch_bounds__(kThreads) k_twostage(const KArgs a) {
     cta_publish_flag(c, ticket);
     if (!block_barrier(a, c, kPhStart)) return;
   }
-  const int64_t stride = static_cast<int64_t>(a.B) * kThreads;
-  const int64_t t0 = static_cast<int64_t>(c.b) * kThreads + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(a.B) * T;
+  const int64_t t0 = static_cast<int64_t>(c.b) * T + threadIdx.x;
   const int64_t piece = (a.items + a.P - 1) / a.P;
   void* own = a.ptr.out[c.r];
   {
