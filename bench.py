@@ -3,26 +3,33 @@
 
 One step = one all-reduce call (VRAR_ALGO_AUTO: the per-size selector plus the
 kernel it picks) over one batch of synthetic input: P = 8 virtual ranks, a
-decode-shaped message of 64 tokens x hidden 8192 bf16 (1 MiB per rank),
-values N(0, 1), seed 0.
+prefill-shaped message of 16,384 tokens x hidden 7168 bf16 (224 MiB per rank,
+1.88 GB of inputs over the 8 ranks), values N(0, 0.02), seed 0: the largest
+workload that fits one GPU, a 16k-token prefill at 8-way tensor parallelism.
 
-Timing: W warm-up steps, then EXACTLY K steps captured as one CUDA graph and
-replayed once between CUDA events on the launching stream, bracketed by a
-barrier and a device synchronise. Consecutive steps rotate through buffer sets
-whose total is more than 3x the L2 size, so every step reads its inputs from
-HBM. busbw = algbw * 2(P-1)/P with algbw = n * bytes-per-element / t (the
-nccl-tests convention). The roofline fraction uses the algorithm-independent
-minimum traffic B_min = 2 * P * n * s (every input read once, every output
-written once) against the measured HBM copy bandwidth.
+Timing: W warm-up steps, then EXACTLY K steps captured as one CUDA graph. The
+graph is replayed R times; each replay is bracketed by a barrier and a device
+synchronise and timed with CUDA events on the launching stream, and the
+reported time per step is the median replay divided by K. Every step reads
+1.88 GB of inputs and writes 1.88 GB of outputs, far more than the 126 MB L2,
+so every step reads its inputs from HBM (smaller shapes rotate through buffer
+sets whose total is more than 3x the L2 size). busbw = algbw * 2(P-1)/P with
+algbw = n * bytes-per-element / t (the nccl-tests convention). The roofline
+fraction uses the algorithm-independent minimum traffic B_min = 2 * P * n * s
+(every input read once, every output written once) against the measured HBM
+copy bandwidth.
 
 Other keys: e2e (same metric with the inputs copied from pinned host memory
 and the outputs copied back inside the timed region), cpu_baseline (the CPU
-oracle on this host), per_algo (each algorithm on the step's workload),
-warm_l2 (the same with one buffer set reused, so the working set stays in L2;
-never the headline) and sweep (the other workload shapes and sizes).
+oracle on one pinned host core, on a contiguous slice of the workload),
+per_algo (each algorithm on the step's workload) and sweep (the other
+workload shapes and sizes: the decode message of 64 tokens x 8192 with its
+warm-L2 and start/end-barrier rows, 128 KiB - 2 MiB per rank with recursive
+doubling timed over graphs of 1000 calls, 2 ranks of small integers, 32 ranks
+as 4 groups of 8, fp16 and fp32 partials on the wire).
 
 --impl reference times the CPU oracle instead (the only reference that exists
-for this method), on bounded samples of the same workload.
+for this method), on bounded slices of the same workload.
 
 Multi-GPU: replicas only. Each rank runs the same single-GPU workload on its
 own device; the time is the maximum over ranks and value sums all ranks' work.
@@ -55,13 +62,24 @@ UNIT = "GB/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 
-WORKLOAD = dict(name="decode 64x8192 bf16, P=8 virtual ranks (1 MiB per rank), N(0,1), seed 0",
-                P=8, n=64 * 8192, dtype="bf16", dist="normal:0,1", seed=0)
+WORKLOAD = dict(name="prefill 16384x7168 bf16, P=8 virtual ranks (224 MiB per rank), N(0,0.02), seed 0",
+                key="prefill_p8_224mib", P=8, n=16384 * 7168, dtype="bf16", dist="normal:0,0.02", seed=0)
+DECODE = dict(name="decode 64x8192 bf16, P=8 virtual ranks (1 MiB per rank), N(0,1), seed 0",
+              P=8, n=64 * 8192, dtype="bf16", dist="normal:0,1", seed=0)
+
+HEADLINE_REPLAYS = 15   # replays of the K-step graph; the median is reported
+SWEEP_REPLAYS = 5
+RD_CALLS = 1000         # recursive doubling rows: graphs of 1000 back-to-back calls (flag reuse)
+PER_ALGO_STEPS = 10     # graph length of the per-algorithm rows on the headline workload
 
 SWEEP = (
-    [dict(name=f"P=8 sweep {b >> 10} KiB per rank, N(0,1)", P=8, n=b // 2, dtype="bf16", dist="normal:0,1",
-          algos=("oneshot", "twostage", "twostage_write", "rd", "auto"), collectives=("rs", "ag")) for b in
-     (128 << 10, 256 << 10, 512 << 10, 1 << 20, 2 << 20)]
+    [dict(DECODE, algos=("oneshot", "twostage", "twostage_write", "rd", "auto"), collectives=("rs", "ag"),
+          warm=("auto", "oneshot", "twostage", "twostage_write", "rd"),
+          edge=("oneshot", "twostage_write"))]
+    + [dict(name=f"P=8 sweep {b >> 10} KiB per rank, N(0,1)", P=8, n=b // 2, dtype="bf16", dist="normal:0,1",
+            algos=("oneshot", "twostage", "twostage_write", "rd", "auto"), collectives=("rs", "ag"),
+            edge=("oneshot", "twostage_write") if b == 2 << 20 else ())
+       for b in (128 << 10, 256 << 10, 512 << 10, 2 << 20)]
     + [dict(name="P=2 ints 128 KiB per rank", P=2, n=65536, dtype="bf16", dist="int8",
             algos=("oneshot", "rd", "auto"))]
     + [dict(name=f"P=32 hier 4x8 {b >> 10} KiB per rank, uniform(-1,1)", P=32, n=b // 2, dtype="bf16",
@@ -73,15 +91,13 @@ SWEEP = (
             dtype="bf16", dist="normal:0,1", algos=("rd",), wire="fp32") for b in (128 << 10, 2 << 20)]
     + [dict(name="P=32 hier 4x8 2048 KiB per rank, uniform(-1,1), fp32 partials on the wire", P=32,
             n=(2 << 20) // 2, dtype="bf16", dist="uniform:-1,1", L=8, algos=("hier",), wire="fp32")]
-    + [dict(name="P=8 prefill 16384x7168 bf16 (224 MiB per rank), N(0,0.02)", P=8, n=16384 * 7168,
-            dtype="bf16", dist="normal:0,0.02", algos=("twostage", "twostage_write", "auto"), steps=20,
-            collectives=("rs", "ag"))]
 )
 
 # The oracle algorithm the reference arm times: the same summation the GPU
 # path's choice for the workload computes (the three custom all-reduce variants
 # share one order, so any of them gives the same bits).
 REFERENCE_ALGO = "twostage_write"
+REFERENCE_SAMPLE = 1 << 21  # elements per rank of each reference step (4 MiB of bf16)
 
 TDT = {"bf16": torch.bfloat16, "fp32": torch.float32, "fp16": torch.float16}
 ESZ = {"bf16": 2, "fp32": 4, "fp16": 2}
@@ -332,30 +348,37 @@ def upload_graph(g) -> bool:
         return False
 
 
-def time_graph(g, world=1, device=None) -> float:
-    """Milliseconds of one replay, timed with events on the launching stream."""
+def time_graph(g, world=1, device=None, replays: int = 1) -> float:
+    """Milliseconds of one replay of a captured graph: the median of `replays`
+    replays, each bracketed by a barrier and a device synchronise and timed
+    with CUDA events on the launching stream."""
     upload_graph(g)
     s = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world, device)
-    torch.cuda.synchronize()
-    e0.record(s)
-    g.replay()
-    e1.record(s)
-    e1.synchronize()
-    torch.cuda.synchronize()
-    barrier(world, device)
-    return e0.elapsed_time(e1)
+    times = []
+    for _ in range(max(1, replays)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world, device)
+        torch.cuda.synchronize()
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        barrier(world, device)
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
 
 
-def measure_algo(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None):
+def measure_algo(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None, replays: int = 1):
+    """Milliseconds per call: a graph of `warmup` calls replayed once, then a
+    graph of `steps` calls timed over `replays` replays (median), max over ranks."""
     wl.call(0, algo, torch.cuda.current_stream().cuda_stream)  # sizes the workspace outside capture
     torch.cuda.synchronize()
     gw = wl.graph(algo, warmup)
     gt = wl.graph(algo, steps, offset=warmup)
     gw.replay()
     torch.cuda.synchronize()
-    ms = max_over_ranks(time_graph(gt, world, device), world, device)
+    ms = max_over_ranks(time_graph(gt, world, device, replays), world, device)
     rc, info = wl.vrar.query_status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} {info} after {algo}")
@@ -363,7 +386,7 @@ def measure_algo(wl: Workload, algo: str, steps: int, warmup: int, world=1, devi
     return ms / steps
 
 
-def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1, device=None):
+def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1, device=None, replays: int = 1):
     """Milliseconds per call of the standalone reduce-scatter ('rs') or
     all-gather ('ag') on the workload's shape (graph of `steps` calls)."""
     wl.collective_call(0, kind, torch.cuda.current_stream().cuda_stream)
@@ -380,7 +403,7 @@ def measure_collective(wl: Workload, kind: str, steps: int, warmup: int, world=1
     gw, gt = graph(warmup, 0), graph(steps, warmup)
     gw.replay()
     torch.cuda.synchronize()
-    ms = max_over_ranks(time_graph(gt, world, device), world, device)
+    ms = max_over_ranks(time_graph(gt, world, device, replays), world, device)
     del gw, gt
     return ms / steps
 
@@ -413,20 +436,25 @@ def entry(wl: Workload, t_s: float, peak: float, algo: str):
 
 def measure_e2e(wl: Workload, algo: str, steps: int, warmup: int, world=1, device=None):
     """Every step copies its P inputs from pinned host memory to the device,
-    runs the all-reduce through the public binding, and copies its P outputs
-    back to pinned host memory. Steps are pipelined the way a user streaming
-    batches would: copies in (one stream), the all-reduce (another) and copies
-    out (a third) of consecutive steps overlap, on two device buffer sets; PCIe
-    carries both directions at once."""
+    runs the all-reduce through the public binding (the C ABI), and copies its
+    P outputs back to pinned host memory. Steps are pipelined the way a user
+    streaming batches would: copies in (one stream), the all-reduce (another)
+    and copies out (a third) of consecutive steps overlap, on two device buffer
+    sets; the host link carries both directions at once."""
     vrar = wl.vrar
     # The P rank buffers of a set are rows of one [P, n] block, so that a step
     # moves its inputs in one copy and its outputs out in one copy.
     dev = wl.base[0].device
-    h_in = torch.stack([t.cpu() for t in wl.base]).pin_memory()
-    h_out = [torch.empty_like(h_in).pin_memory() for _ in range(2)]
+    shape, dtype = (wl.P, wl.n), wl.base[0].dtype
+    h_in = torch.empty(shape, dtype=dtype, pin_memory=True)
+    for p, t in enumerate(wl.base):
+        h_in[p].copy_(t)
+    # One host output block: the copies out are ordered on their own stream,
+    # and nothing reads the host copy inside the timed region.
+    h_out = torch.empty(shape, dtype=dtype, pin_memory=True)
     sets = 2
-    d_in_blk = [torch.empty(h_in.shape, dtype=h_in.dtype, device=dev) for _ in range(sets)]
-    d_out_blk = [torch.empty(h_in.shape, dtype=h_in.dtype, device=dev) for _ in range(sets)]
+    d_in_blk = [torch.empty(shape, dtype=dtype, device=dev) for _ in range(sets)]
+    d_out_blk = [torch.empty(shape, dtype=dtype, device=dev) for _ in range(sets)]
     d_in = [list(blk.unbind(0)) for blk in d_in_blk]
     d_out = [list(blk.unbind(0)) for blk in d_out_blk]
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
@@ -449,7 +477,7 @@ def measure_e2e(wl: Workload, algo: str, steps: int, warmup: int, world=1, devic
         run_done[b].record(s_run)
         s_out.wait_event(run_done[b])
         with torch.cuda.stream(s_out):
-            h_out[b].copy_(d_out_blk[b], non_blocking=True)
+            h_out.copy_(d_out_blk[b], non_blocking=True)
         out_done[b].record(s_out)
 
     for i in range(warmup):
@@ -467,38 +495,131 @@ def measure_e2e(wl: Workload, algo: str, steps: int, warmup: int, world=1, devic
     torch.cuda.synchronize()
     barrier(world, device)
     ms = max_over_ranks(e0.elapsed_time(e1), world, device) / steps
+    # The last step's outputs are on the host: check one rank against another.
+    if not torch.equal(h_out[0].view(torch.int16), h_out[wl.P - 1].view(torch.int16)):
+        raise RuntimeError("e2e: rank outputs differ after the copy back")
     bytes_in = h_in.numel() * h_in.element_size()
-    bytes_out = h_out[0].numel() * h_out[0].element_size()
-    del d_in_blk, d_out_blk
+    bytes_out = h_out.numel() * h_out.element_size()
+    del d_in_blk, d_out_blk, d_in, d_out, h_in, h_out
     return ms, bytes_in, bytes_out
 
 
 # ---- CPU oracle timing ----------------------------------------------------------------------------
 
-def oracle_samples(spec, algo: str, min_seconds: float, n_sample: int | None = None, max_calls=None):
-    """Time the CPU oracle on the workload (or a contiguous slice of n_sample
-    elements per rank); returns (seconds per full-size call, calls, sample text)."""
+def host_description() -> dict:
+    """Host facts reported beside the CPU oracle's time."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        allowed = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        allowed = None
+    return {"nproc": os.cpu_count(), "cpus_allowed": allowed, "cpu_model": model}
+
+
+class one_core:
+    """Pin this process to one of its allowed cores for the duration (the
+    oracle is single-threaded; pinning keeps it from migrating)."""
+
+    def __enter__(self):
+        self.old = None
+        self.core = None
+        try:
+            self.old = os.sched_getaffinity(0)
+            self.core = min(self.old)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            self.old = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.old is not None:
+            os.sched_setaffinity(0, self.old)
+
+    def describe(self) -> str:
+        return f"os.sched_setaffinity to core {self.core}" if self.core is not None else "not pinned"
+
+
+def oracle_inputs(spec, n_sample: int, device=None):
+    """The first n_sample elements of every rank's input of the workload (the
+    counter-based generator gives the same values as the full-size buffers),
+    as numpy arrays for the oracle."""
+    P, dt = spec["P"], spec["dtype"]
+    m = min(spec["n"], n_sample)
+    xs = synth.make_inputs(P, m, TDT[dt], synth.parse_dist(spec["dist"]), seed=spec.get("seed", 0),
+                           device=device or "cpu", block=1 << 24)
+    return [t.cpu().view(torch.int16).numpy().view(np.uint16) if dt != "fp32" else t.cpu().numpy() for t in xs], m
+
+
+def oracle_samples(spec, algo: str, min_seconds: float, n_sample: int, device=None):
+    """Time the CPU oracle, pinned to one core, on a contiguous slice of
+    n_sample elements per rank of the workload; returns (seconds per full-size
+    call scaled by n / n_sample, calls, sample text, host facts)."""
     import oracle
     P, n, dt = spec["P"], spec["n"], spec["dtype"]
-    m = n if n_sample is None else min(n, n_sample)
-    xs = synth.make_inputs(P, m, TDT[dt], synth.parse_dist(spec["dist"]), seed=spec.get("seed", 0))
-    xs = [t.view(torch.int16).numpy().view(np.uint16) if dt == "bf16" else t.numpy() for t in xs]
+    xs, m = oracle_inputs(spec, n_sample, device)
     L = spec.get("L", 8)
     oracle.allreduce(algo, xs, dt, L=L)  # builds/loads the library outside the timing
-    calls, t0 = 0, time.perf_counter()
-    while True:
-        oracle.allreduce(algo, xs, dt, L=L)
-        calls += 1
-        el = time.perf_counter() - t0
-        if el >= min_seconds or (max_calls and calls >= max_calls):
-            break
+    with one_core() as pin:
+        calls, t0 = 0, time.perf_counter()
+        while True:
+            oracle.allreduce(algo, xs, dt, L=L)
+            calls += 1
+            el = time.perf_counter() - t0
+            if el >= min_seconds:
+                break
     per_call = el / calls * (n / m)
     sample = f"{calls} oracle calls of '{algo}' on {P} x {m} {dt} elements" + \
-             ("" if m == n else f" (a contiguous slice; time scaled by {n}/{m})")
-    return per_call, calls, sample
+             ("" if m == n else f" (the first {m} elements of every rank; time scaled by {n}/{m})")
+    return per_call, calls, sample, dict(host_description(), affinity=pin.describe(), threads=1)
 
 
 # ---- arms -------------------------------------------------------------------------------------------
+
+def with_edge(algo: str):
+    """'twostage_write+edge' -> ('twostage_write', True): the algorithm with the
+    start/end barriers on."""
+    return (algo[:-5], True) if algo.endswith("+edge") else (algo, False)
+
+
+def measure_row(vrar, w: Workload, algo: str, steps: int, warmup: int, world, device, replays: int):
+    base, edge = with_edge(algo)
+    vrar.set_edge_sync(edge)  # read when a call is queued: the graph keeps it
+    try:
+        return measure_algo(w, base, steps, warmup, world, device, replays)
+    finally:
+        vrar.set_edge_sync(False)
+
+
+def spin_row(vrar, w: Workload, algo: str, calls: int) -> dict:
+    """Spin statistics of the waits of `calls` calls (a separate, instrumented
+    graph: the counters cost a few atomics per warp and wait, so the timed rows
+    run without them)."""
+    base, edge = with_edge(algo)
+    vrar.set_edge_sync(edge)
+    vrar.set_spin_stats(True)
+    try:
+        w.call(0, base, torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        g = w.graph(base, calls)
+        vrar.get_spin_stats(reset=True)
+        g.replay()
+        torch.cuda.synchronize()
+    finally:
+        vrar.set_spin_stats(False)
+        vrar.set_edge_sync(False)
+    st = vrar.get_spin_stats(reset=True)
+    rc, _ = vrar.query_status()
+    del g
+    return {"calls": calls, "status": rc, **st}
+
 
 def run_vrar(args):
     import collective_all_reduce_virtual_b200 as vrar
@@ -517,9 +638,9 @@ def run_vrar(args):
     wl = Workload(WORKLOAD, device)
     algo_auto = vrar.select_algo(wl.P, wl.n, TDT[wl.dt])
 
-    # The timed steps: exactly K AUTO calls.
+    # The timed steps: exactly K AUTO calls per graph replay, median of R replays.
     with nvtx("timed steps"):
-        t_step_ms = measure_algo(wl, "auto", args.steps, args.warmup, world, device)
+        t_step_ms = measure_algo(wl, "auto", args.steps, args.warmup, world, device, args.replays)
     t_s = t_step_ms / 1e3
 
     # e2e through the public call with host buffers.
@@ -529,17 +650,16 @@ def run_vrar(args):
     per_algo = {}
     if not args.quick:
         for algo in ("oneshot", "twostage", "twostage_write", "rd"):
-            per_algo[algo] = entry(wl, measure_algo(wl, algo, 200, 5, world, device) / 1e3, peak, algo)
+            per_algo[algo] = entry(wl, measure_algo(wl, algo, PER_ALGO_STEPS, 3, world, device, 3) / 1e3, peak,
+                                   algo)
+        for kind in ("rs", "ag"):
+            t = measure_collective(wl, kind, PER_ALGO_STEPS, 3, world, device, 3) / 1e3
+            ach = (wl.P + 1) * wl.n * wl.esz / t / 1e9  # (P + 1) n s either way
+            per_algo["reduce_scatter" if kind == "rs" else "all_gather"] = {
+                "us": round(t * 1e6, 3), "hbm_gbs": round(ach, 1), "frac": round(ach / peak, 4)}
     wl.free()
-
-    # Warm L2: the same buffers every call (inputs and outputs, 16 MiB, stay in
-    # the 126 MB L2). Reported beside the cold numbers, never as the headline.
-    warm = {}
-    if not args.quick:
-        ww = Workload(WORKLOAD, device, rotate=False)
-        for algo in ("auto", "oneshot", "twostage", "twostage_write", "rd"):
-            warm[algo] = entry(ww, measure_algo(ww, algo, 200, 5, world, device) / 1e3, peak, algo)
-        ww.free()
+    del wl
+    torch.cuda.empty_cache()
 
     sweep = []
     if not args.quick:
@@ -552,15 +672,29 @@ def run_vrar(args):
                    "selected": vrar.select_algo(w.P, w.n, TDT[w.dt]),
                    "kernel": vrar.kernel_name(w.P, w.n, TDT[w.dt], "auto")}
             for algo in spec["algos"]:
-                k = spec.get("steps", 200)
-                row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device) / 1e3, peak, algo)
+                k = RD_CALLS if algo == "rd" else spec.get("steps", 200)
+                row[algo] = entry(w, measure_algo(w, algo, k, 3, world, device, SWEEP_REPLAYS) / 1e3, peak, algo)
+                if algo == "rd":
+                    row[algo]["calls_per_graph"] = k
+            for algo in spec.get("edge", ()):
+                key = f"{algo}+edge"
+                row[key] = entry(w, measure_row(vrar, w, key, 200, 3, world, device, SWEEP_REPLAYS) / 1e3, peak,
+                                 algo)
+                row[key]["spin"] = spin_row(vrar, w, key, 1000)
             for kind in spec.get("collectives", ()):
                 # RS moves P*n*s in and n*s out; AG n*s in and P*n*s out: (P+1)*n*s either way.
-                t = measure_collective(w, kind, spec.get("steps", 200), 3, world, device) / 1e3
+                t = measure_collective(w, kind, spec.get("steps", 200), 3, world, device, SWEEP_REPLAYS) / 1e3
                 ach = (w.P + 1) * w.n * w.esz / t / 1e9
                 row["reduce_scatter" if kind == "rs" else "all_gather"] = {
                     "us": round(t * 1e6, 3), "hbm_gbs": round(ach, 1), "frac": round(ach / peak, 4)}
             w.free()
+            if spec.get("warm"):
+                # The same buffers every call: the working set stays in L2. Beside the
+                # cold numbers, never the headline.
+                ww = Workload(spec, device, rotate=False)
+                row["warm_l2"] = {a: entry(ww, measure_algo(ww, a, 200, 3, world, device, SWEEP_REPLAYS) / 1e3,
+                                           peak, a) for a in spec["warm"]}
+                ww.free()
             torch.cuda.empty_cache()
             vrar.set_group_size(8)
             vrar.set_payload_wire("element")
@@ -573,17 +707,19 @@ def run_vrar(args):
     value = world * busbw_gbs(P, n, esz, t_s)
     achieved = b_min_bytes(P, n, esz) / t_s / 1e9
     kernel = vrar.kernel_name(P, n, TDT[WORKLOAD["dtype"]], "auto")
-    traffic, traffic_src = profiled_traffic(kernel, "decode_p8_1mib")
+    traffic, traffic_src = profiled_traffic(kernel, WORKLOAD["key"])
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step_ms, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD["name"], "P": P, "n": n, "algo": f"auto -> {algo_auto}",
-                   "l2": f"inputs rotate through {rotation_sets(b_min_bytes(P, n, esz))} buffer sets "
-                         f"({rotation_sets(b_min_bytes(P, n, esz)) * b_min_bytes(P, n, esz) >> 20} MiB) "
-                         f"> 3x the 126 MB L2",
-                   "timing": "K calls captured in one CUDA graph, replayed once between CUDA events",
+                   "l2": f"inputs larger than L2: every step reads {P * n * esz / 1e9:.2f} GB of inputs and "
+                         f"writes as much, against the 126 MB L2",
+                   "timing": f"K = {args.steps} calls captured in one CUDA graph; the graph replayed "
+                             f"R = {args.replays} times, each replay bracketed by a barrier and a device "
+                             f"synchronise and timed with CUDA events on the launching stream; "
+                             f"ms_per_step = median replay / K",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, P virtual ranks"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -593,18 +729,18 @@ def run_vrar(args):
                      "traffic_source": traffic_src},
         "e2e": {"value": round(world * busbw_gbs(P, n, esz, e2e_ms / 1e3), 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * args.replays,
+        "gpu_launches_note": "one kernel per step: K steps in each of the R timed replays",
         "clocks": clk,
         "per_algo": per_algo,
-        "warm_l2": {"note": "same buffers every call (working set in L2); not the headline, which is cold",
-                    **warm} if warm else None,
         "sweep": sweep,
     }
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_call, calls, sample = oracle_samples(WORKLOAD, algo_auto, min_seconds=args.cpu_seconds)
+        per_call, calls, sample, host = oracle_samples(WORKLOAD, algo_auto, min_seconds=args.cpu_seconds,
+                                                       n_sample=args.cpu_sample, device=device)
         line["cpu_baseline"] = {"value": round(busbw_gbs(P, n, esz, per_call), 4), "unit": UNIT, "cores": 1,
-                                "kind": "oracle", "sample": sample}
+                                "kind": "oracle", "sample": sample, **host}
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -612,30 +748,34 @@ def run_vrar(args):
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on one pinned host core.
+    Each step is the oracle on a contiguous slice of the workload (the first
+    REFERENCE_SAMPLE elements of every rank); busbw is scaled to the full size."""
     rank, world, _ = dist_env()
     if rank != 0:
         return None
+    import oracle
     P, n, esz = WORKLOAD["P"], WORKLOAD["n"], ESZ[WORKLOAD["dtype"]]
     algo = REFERENCE_ALGO
-    n_sample = 65536
-    import oracle
-    xs = synth.make_inputs(P, n_sample, TDT[WORKLOAD["dtype"]], synth.parse_dist(WORKLOAD["dist"]), seed=0)
-    xs = [t.view(torch.int16).numpy().view(np.uint16) for t in xs]
-    for _ in range(args.warmup):
-        oracle.allreduce(algo, xs, "bf16")
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.allreduce(algo, xs, "bf16")
-    el = time.perf_counter() - t0
-    per_full = el / args.steps * (n / n_sample)
+    xs, m = oracle_inputs(WORKLOAD, REFERENCE_SAMPLE)
+    oracle.allreduce(algo, xs, "bf16")  # loads the library
+    with one_core() as pin:
+        for _ in range(args.warmup):
+            oracle.allreduce(algo, xs, "bf16")
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle.allreduce(algo, xs, "bf16")
+        el = time.perf_counter() - t0
+    per_full = el / args.steps * (n / m)
     v = busbw_gbs(P, n, esz, per_full)
-    sample = (f"each step: oracle '{algo}' on a {P} x {n_sample} bf16 slice of the workload; "
-              f"time scaled by {n}/{n_sample}")
+    sample = (f"each step: oracle '{algo}' on the first {m} elements of each of the {P} ranks of the workload; "
+              f"time scaled by {n}/{m}")
     return {"metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "reference",
             "config": {"workload": WORKLOAD["name"], "P": P, "n": n, "algo": algo},
-            "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                             **host_description(), "affinity": pin.describe(), "threads": 1},
             "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -650,7 +790,7 @@ def run_selector_sweep(args):
     kernel = os.environ.get("VRAR_WRITE_KERNEL", "auto")
     for P in (2, 4, 8, 16, 32):
         for kib in (32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384):
-            spec = dict(WORKLOAD, P=P, n=kib * 512, name=f"P={P} {kib} KiB per rank")
+            spec = dict(DECODE, P=P, n=kib * 512, name=f"P={P} {kib} KiB per rank")
             wl = Workload(spec, device)
             row = {"P": P, "kib": kib, "write_kernel": kernel, "selected": vrar.select_algo(P, wl.n, TDT[wl.dt]),
                    "kernel": vrar.kernel_name(P, wl.n, TDT[wl.dt], "auto")}
@@ -677,7 +817,7 @@ def run_case(spec_text: str):
     calls = int(parts[3]) if len(parts) > 3 else 6
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    wl = Workload(dict(WORKLOAD, P=P, n=kib * 512, name=spec_text), device)
+    wl = Workload(dict(DECODE, P=P, n=kib * 512, name=spec_text), device)
     h = torch.cuda.current_stream().cuda_stream
     for i in range(calls):
         if algo in ("rs", "ag"):
@@ -692,12 +832,12 @@ def run_case(spec_text: str):
 
 def run_spin_stats(args):
     """Spin statistics of the cross-rank waits over many calls (JSON lines):
-    for each algorithm with waits, `--spin-stats N` calls on the step's
-    workload, as graphs of 1000 calls."""
+    for each algorithm with waits, `--spin-stats N` calls on the decode
+    workload (8 ranks x 1 MiB), as graphs of 1000 calls."""
     import collective_all_reduce_virtual_b200 as vrar
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    wl = Workload(WORKLOAD, device)
+    wl = Workload(DECODE, device)
     per = 1000
     for algo, edge in (("twostage", False), ("twostage_write", True), ("rd", False)):
         vrar.set_edge_sync(edge)
@@ -835,7 +975,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("vrar", "reference"), default="vrar")
     ap.add_argument("--quick", action="store_true", help="skip the per-algorithm table and the sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--replays", type=int, default=HEADLINE_REPLAYS,
+                    help="timed replays of the K-step graph (the median is reported)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 23,
+                    help="elements per rank of the slice the CPU oracle baseline runs on")
     ap.add_argument("--case", metavar="ALGO,P,KIB[,CALLS]",
                     help="run a few calls of one algorithm on one shape and exit (for profilers)")
     ap.add_argument("--spin-stats", type=int, metavar="CALLS", default=0,

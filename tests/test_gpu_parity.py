@@ -225,33 +225,6 @@ def test_config_p32_hier_4x8(n):
     assert_bits(got, oracle.allreduce("hier", xs, "bf16", L=8), f"hier 4x8 n={n}")
 
 
-@pytest.mark.slow
-def test_config_p8_prefill_sampled():
-    """16384 x 7168 bf16 per rank (1.88 GB of inputs): the 2-stage kernels on the
-    full size, checked on sampled outputs (every output element depends only on
-    the P inputs at the same index) and for equality of all P outputs."""
-    P, n = 8, 16384 * 7168
-    d_in = synth.make_inputs(P, n, torch.bfloat16, synth.normal(0.0, 0.02), seed=0, device="cuda",
-                             block=1 << 25)
-    rng = np.random.default_rng(0)
-    piece = (n // 8 + P - 1) // P * 8
-    edges = np.concatenate([np.arange(0, 64), n - 64 + np.arange(64)] +
-                           [np.arange(s * piece - 8, s * piece + 8) for s in range(1, P)])
-    idx = np.unique(np.concatenate([rng.integers(0, n, 200_000), edges]))
-    idx_t = torch.from_numpy(idx).cuda()
-    xs_s = [to_np(t[idx_t]) for t in d_in]
-    for algo in ("twostage", "twostage_write"):
-        outs = vrar.all_reduce(d_in, algo=algo)
-        rc, info = vrar.query_status()
-        assert rc == 0, info
-        want = oracle.allreduce(algo, xs_s, "bf16")
-        assert_bits([to_np(o[idx_t]) for o in outs], want, f"{algo} sampled")
-        for p in range(1, P):
-            assert torch.equal(outs[p].view(torch.int16), outs[0].view(torch.int16)), f"{algo} rank {p}"
-        del outs
-    torch.cuda.empty_cache()
-
-
 # ---- protocol properties ----------------------------------------------------------------------
 
 @pytest.mark.parametrize("algo", ["oneshot", "twostage", "twostage_write", "rd", "hier"])
@@ -499,3 +472,74 @@ def test_allreduce_overlapped_with_gemm_on_another_stream():
         parts = [to_np(p.reshape(-1)[idx]) for p in m.part[u]]
         want = oracle.allreduce(vrar.select_algo(m.P, m.T * m.H), parts, "bf16")
         assert_bits([to_np(o.reshape(-1)[idx]) for o in m.out[u]], want, f"micro-batch {u}")
+
+
+# ---- first use of the workspace, and its size ---------------------------------------------------
+
+FIRST_CALL = """
+import sys
+sys.path[:0] = [{root!r}, {tests!r}]
+import numpy as np
+import torch
+import collective_all_reduce_virtual_b200 as vrar
+import oracle, synth
+from util import from_np, gen, to_np
+
+side = torch.cuda.Stream()  # created non-blocking: not ordered with the legacy default stream
+for algo, P, n in (("rd", 8, 300_001), ("twostage", 8, 300_001), ("hier", 8, 200_003)):
+    xs = gen(P, n, "bf16", synth.normal(0.0, 1.0), seed=P + n)
+    d_in = [from_np(x, "bf16").cuda() for x in xs]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        outs = vrar.all_reduce(d_in, algo=algo, stream=side)
+    side.synchronize()
+    rc, info = vrar.query_status()
+    assert rc == 0, (algo, rc, info)
+    want = oracle.allreduce(algo, xs, "bf16", L=8)
+    for p in range(P):
+        assert np.array_equal(to_np(outs[p]), want[p]), (algo, p)
+print("ok")
+"""
+
+
+def test_first_calls_of_a_process_on_a_side_stream():
+    """The workspace is allocated and zeroed by the first call that needs it;
+    that call may come on a non-blocking stream, which is not ordered with the
+    zeroing by stream semantics, so the zeroing must be complete before it
+    returns. A fresh process makes first calls of three algorithms there (the
+    first allocates the control words and the slots, the third grows the
+    slots)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = FIRST_CALL.format(root=root, tests=os.path.join(root, "tests"))
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0 and "ok" in res.stdout, res.stdout[-2000:] + res.stderr[-4000:]
+
+
+def test_payload_slots_are_bounded_by_the_grid():
+    """Recursive doubling and the hierarchical algorithm reuse their payload
+    slots round by round once the grid cannot cover the message in one round,
+    so their slot bytes stop growing with the message."""
+    one_round = lambda P, items, steps: P * steps * items * 32  # noqa: E731
+    # 8 x 128 KiB: one round, one slot per item
+    assert vrar.workspace_bytes(8, 65_536, torch.bfloat16, "rd") == one_round(8, 8192, 3)
+    big = [vrar.workspace_bytes(8, n, torch.bfloat16, "rd") for n in (1 << 22, 1 << 24, 16384 * 7168)]
+    assert big[0] == big[1] == big[2], big
+    assert big[2] < one_round(8, (16384 * 7168) // 8, 3) // 100, big
+    assert big[2] <= 64 << 20, big
+    h = [vrar.workspace_bytes(32, n, torch.bfloat16, "hier") for n in (1 << 22, 1 << 24)]
+    assert h[0] == h[1] and h[1] <= 64 << 20, h
+    # the full-size prefill through recursive doubling, against the oracle on sampled windows
+    P, n = 8, 16384 * 7168
+    d_in = synth.make_inputs(P, n, torch.bfloat16, synth.normal(0.0, 0.02), seed=0, device="cuda", block=1 << 25)
+    outs = vrar.all_reduce(d_in, algo="rd")
+    rc, info = vrar.query_status()
+    assert rc == 0, info
+    for lo in (0, n // 3 - 4096, n - 8192):
+        xs = [to_np(t[lo:lo + 8192]) for t in d_in]
+        want = oracle.allreduce("rd", xs, "bf16")
+        assert_bits([to_np(o[lo:lo + 8192]) for o in outs], want, f"rd prefill window {lo}")
+    del outs, d_in
+    torch.cuda.empty_cache()
