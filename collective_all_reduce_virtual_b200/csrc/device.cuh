@@ -74,6 +74,8 @@ struct KArgs {
   uint32_t* ctrl;
   uint32_t* sig;     // kPhases x kSigPhaseWords flag words
   uint64_t* ll;      // payload slots
+  int64_t slot_items;  // payload slots (32 bytes each) per rank, step and slot set
+  int slot_sets;       // 1: slot = item index (one round); 2: slots reused by round parity
   unsigned long long* stats;  // spin statistics, or null when they are off
 };
 
@@ -427,10 +429,13 @@ __device__ __forceinline__ void prefetch_items(const void* base, int64_t first, 
 // serialises the adds). The CTA that sees the low half reach gridDim.x - 1 is
 // the last to arrive, and adds 2^32 - gridDim.x: the call count goes up by one
 // and the arrival count back to 0, for the next launch (stream order). Every
-// CTA of a call therefore reads the same call count c and uses c + 1 as the
-// call's flag; flags grow by one per call that uses them, so a flag or payload
-// word left by any earlier call never equals the current flag (until 2^32
-// calls wrap it). Kernels that use no flags never touch the ticket.
+// CTA of a call therefore reads the same call count c and uses
+// (c mod (2^31 - 1)) + 1 as the call's flag: never 0 (the value of a
+// never-written word) and below 2^31, so that payload tags can carry a lap bit
+// in bit 31 (see rd_tag). Flags grow by one per call that uses them, so a flag
+// or payload word left by any earlier call never equals the current flag
+// (until 2^31 - 1 calls wrap it). Kernels that use no flags never touch the
+// ticket.
 
 struct Cta {
   int r;          // virtual rank this CTA acts for
@@ -461,10 +466,7 @@ __device__ __forceinline__ unsigned long long cta_take_ticket(const KArgs& a) {
 // Broadcast the call's flag to the whole CTA (contains a CTA barrier).
 __device__ __forceinline__ void cta_publish_flag(Cta& c, unsigned long long ticket) {
   __shared__ uint32_t s_flag;
-  if (threadIdx.x == 0) {
-    const uint32_t f = static_cast<uint32_t>(ticket >> 32) + 1u;
-    s_flag = f == 0u ? 1u : f;  // 0 is the value of a never-written word
-  }
+  if (threadIdx.x == 0) s_flag = static_cast<uint32_t>(ticket >> 32) % 0x7FFFFFFFu + 1u;
   __syncthreads();
   c.flag = s_flag;
 }

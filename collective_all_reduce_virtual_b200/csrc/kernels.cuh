@@ -364,9 +364,35 @@ __global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
 // partner rank XOR 2^s without waiting, then takes the partner's items from its
 // own slot as they arrive and keeps rnd(own + partner).
 //
-// Payload slots: rank q's slot for step s is `per_rank` items of 32 bytes at
-// ll + ((q * steps + s) * per_rank) * 4 words. No slot is ever cleared: a
-// word belongs to this call only if its high half equals the call's flag.
+// A call covers its items in rounds of B*T threads per rank (T = kThreads):
+// in round t, thread t0 of a rank holds items k*per_chunk + t*B*T + t0. Every
+// rank runs the same split, so a thread only ever exchanges with the thread
+// at the same position in its partner rank.
+//
+// Payload slots. A slot is 32 bytes (one item as four 8-byte words). Rank q
+// receives its step-s words in `slot_items` slots of slot set `set`, at
+//   ll + (((set * P + q) * steps + s) * slot_items + slot) * 4 words.
+// When the grid covers the message in one round (slot_sets == 1) the slot of
+// an item is its index. Otherwise (slot_sets == 2) piece k of thread t0 uses
+// slot k*B*T + t0 in every round, in slot set (round & 1): the slots are bound
+// by the grid, not by the message, so they stay in L2 however long the
+// message is. A slot is written again two rounds later, and only after its
+// reader has read it: the writer q reaches round t+2 only after finishing
+// round t+1, whose step s needed the reader p's round-(t+1) word, which p
+// sends only after it has finished round t (and so read its round-t slot).
+// The tag of round t is the call's flag with bit 31 set to bit 1 of t (rd_tag),
+// so a word left from round t-2 never passes for round t's. No slot is ever
+// cleared: a word belongs to this round only if its high half equals the tag.
+
+// Tag of round `rnd` of a call with flag f (f < 2^31, never 0).
+__device__ __forceinline__ uint32_t rd_tag(uint32_t f, int64_t rnd) {
+  return f | (static_cast<uint32_t>((rnd >> 1) & 1) << 31);
+}
+
+// Slot of piece k of thread t0 (item idx) in a round, per the layout above.
+__device__ __forceinline__ int64_t rd_slot(const KArgs& a, int k, int64_t idx, int64_t t0, int64_t stride) {
+  return a.slot_sets == 1 ? idx : k * stride + t0;
+}
 
 // Partner of rank r at step s. Flat RD: r XOR 2^s. Hierarchical (r = g*L + l):
 // the rank holding the same slice l in group g XOR 2^s.
@@ -378,28 +404,27 @@ __device__ __forceinline__ int rd_partner(int r, int s, int L) {
 }
 
 template <class D, int C, bool kHier>
-__device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 (&v)[C], const int64_t (&idx)[C],
-                                            const bool (&val)[C], int64_t per_rank) {
+__device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 (&v)[C], const int64_t (&slot)[C],
+                                            const bool (&val)[C], int set, uint32_t tag) {
   const bool mute = (a.fault_mask >> c.r) & 1u;
-  const uint32_t f = c.flag;
   for (int s = 0; s < a.steps; ++s) {
     const int q = rd_partner<kHier>(c.r, s, a.L);
-    uint64_t* dst = a.ll + (static_cast<size_t>(q) * a.steps + s) * per_rank * 4;
-    const uint64_t* src = a.ll + (static_cast<size_t>(c.r) * a.steps + s) * per_rank * 4;
+    uint64_t* dst = a.ll + ((static_cast<size_t>(set) * a.P + q) * a.steps + s) * a.slot_items * 4;
+    const uint64_t* src = a.ll + ((static_cast<size_t>(set) * a.P + c.r) * a.steps + s) * a.slot_items * 4;
     if (!mute) {
 #pragma unroll
       for (int k = 0; k < C; ++k)
-        if (val[k]) send_item(dst + idx[k] * 4, v[k], f);
+        if (val[k]) send_item(dst + slot[k] * 4, v[k], tag);
     }
     // Poll all C slots together (one L2 round trip per attempt, not C), then
-    // re-poll only the items whose four words do not all carry the flag yet.
+    // re-poll only the items whose four words do not all carry the tag yet.
     uint64_t w[C][4];
     uint32_t pending = 0;
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       if (val[k]) {
-        ld_payload2(src + idx[k] * 4, w[k][0], w[k][1]);
-        ld_payload2(src + idx[k] * 4 + 2, w[k][2], w[k][3]);
+        ld_payload2(src + slot[k] * 4, w[k][0], w[k][1]);
+        ld_payload2(src + slot[k] * 4 + 2, w[k][2], w[k][3]);
         pending |= 1u << k;
       }
     }
@@ -408,13 +433,13 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
     for (;; ++it) {
 #pragma unroll
       for (int k = 0; k < C; ++k)
-        if (((pending >> k) & 1u) && (w[k][0] >> 32) == f && (w[k][1] >> 32) == f && (w[k][2] >> 32) == f &&
-            (w[k][3] >> 32) == f)
+        if (((pending >> k) & 1u) && (w[k][0] >> 32) == tag && (w[k][1] >> 32) == tag && (w[k][2] >> 32) == tag &&
+            (w[k][3] >> 32) == tag)
           pending &= ~(1u << k);
       if (!pending) break;
       if ((it & 15u) == 15u) {
         if (t0 == 0) t0 = globaltimer_ns();
-        if (ld_relaxed(a.ctrl + kFailEpoch) == f) {
+        if (ld_relaxed(a.ctrl + kFailEpoch) == c.flag) {
           record_spins(a, it + 1, false);
           return false;
         }
@@ -427,8 +452,8 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
 #pragma unroll
       for (int k = 0; k < C; ++k) {
         if ((pending >> k) & 1u) {
-          ld_payload2(src + idx[k] * 4, w[k][0], w[k][1]);
-          ld_payload2(src + idx[k] * 4 + 2, w[k][2], w[k][3]);
+          ld_payload2(src + slot[k] * 4, w[k][0], w[k][1]);
+          ld_payload2(src + slot[k] * 4 + 2, w[k][2], w[k][3]);
         }
       }
     }
@@ -443,6 +468,20 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
     }
   }
   return true;
+}
+
+// L2 prefetch of the items CTA b of a rank reads in the round after the one
+// at `base` (T items of each of the C chunks of [lo, lo + len)), issued by
+// threads 0..C-1 while this round's exchange runs.
+template <class D, int C>
+__device__ __forceinline__ void prefetch_next_round(const void* in, int64_t lo, int64_t len, int64_t per_chunk,
+                                                    int64_t base, int64_t stride, int b, int64_t n) {
+  if (threadIdx.x < C) {
+    const int64_t k = threadIdx.x;
+    const int64_t first = base + stride + static_cast<int64_t>(b) * kThreads;
+    const int64_t end = min((k + 1) * per_chunk, len) - k * per_chunk;
+    if (first < end) prefetch_items<D>(in, lo + k * per_chunk + first, min(static_cast<int64_t>(kThreads), end - first), n);
+  }
 }
 
 template <class D, int C>
@@ -462,20 +501,24 @@ __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
   bool ok = true;
   // The trip count is the same for every thread of the CTA (the flag is
   // published inside the first trip, after that trip's input loads issue).
-  for (int64_t base = 0; base < per_chunk; base += stride) {
+  int64_t rnd = 0;
+  for (int64_t base = 0; base < per_chunk; base += stride, ++rnd) {
     const int64_t j = base + t0;
     uint4 v[C];
-    int64_t idx[C];
+    int64_t idx[C], slot[C];
     bool val[C];
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       idx[k] = k * per_chunk + j;
+      slot[k] = rd_slot(a, k, idx[k], t0, stride);
       val[k] = ok && j < per_chunk && idx[k] < a.items;
       if (val[k]) v[k] = load_item_input<D>(a.ptr.in[c.r], idx[k], a.n);
     }
     if (base == 0) cta_publish_flag(c, ticket);
     if (!ok) continue;
-    ok = rd_exchange<D, C, false>(a, c, v, idx, val, a.items);
+    prefetch_next_round<D, C>(a.ptr.in[c.r], 0, a.items, per_chunk, base, stride, c.b, a.n);
+    ok = rd_exchange<D, C, false>(a, c, v, slot, val, a.slot_sets == 1 ? 0 : static_cast<int>(rnd & 1),
+                                  rd_tag(c.flag, rnd));
     if (ok) {
 #pragma unroll
       for (int k = 0; k < C; ++k)
@@ -490,9 +533,10 @@ __global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
 // ascending order, one rounding. Phase 2 (inter-group recursive doubling):
 // log2 G steps of fused-payload exchange with partner (g XOR 2^s, l). Phase 3
 // (in-group all-gather): rank (g, l) streams slice l into the outputs of all
-// L ranks of group g. Slices are cut into C chunks as in k_rd. kMinBlocks 2
-// limits registers to fit two CTAs per SM (more threads in flight when a call
-// needs several rounds over its items).
+// L ranks of group g. Slices are cut into C chunks, and payload slots laid out
+// by round, as in k_rd (item indices are relative to the slice; partners hold
+// the same slice). kMinBlocks 2 limits registers to fit two CTAs per SM (more
+// threads in flight when a call needs several rounds over its items).
 template <class D, int C, int kMinBlocks = 1>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) k_hier(const KArgs a) {
   pdl_trigger();
@@ -512,20 +556,23 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_hier(const KArgs a) {
   pdl_wait();
   const unsigned long long ticket = cta_take_ticket(a);
   bool ok = true;
-  for (int64_t base = 0; base < per_chunk; base += stride) {  // same trip count in the whole CTA
+  int64_t rnd = 0;
+  for (int64_t base = 0; base < per_chunk; base += stride, ++rnd) {  // same trip count in the whole CTA
     const int64_t j = base + t0;
     uint4 v[C];
-    int64_t idx[C];
+    int64_t idx[C], slot[C];
     bool val[C];
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       idx[k] = k * per_chunk + j;
+      slot[k] = rd_slot(a, k, idx[k], t0, stride);
       val[k] = ok && j < per_chunk && idx[k] < len;
       if (val[k]) v[k] = reduce_item<D>(a.ptr, g * L, L, lo + idx[k], a.n);
     }
     if (base == 0) cta_publish_flag(c, ticket);
     if (!ok) continue;
-    ok = rd_exchange<D, C, true>(a, c, v, idx, val, piece);
+    ok = rd_exchange<D, C, true>(a, c, v, slot, val, a.slot_sets == 1 ? 0 : static_cast<int>(rnd & 1),
+                                 rd_tag(c.flag, rnd));
     if (ok) {
 #pragma unroll
       for (int k = 0; k < C; ++k) {
@@ -543,8 +590,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_hier(const KArgs a) {
 // the wire (16-bit element types). Each 16-byte input item becomes two fp32
 // quads that travel as fused payload words exactly like fp32 elements (so
 // twice the payload words of the element-type wire); the steps add in fp32
-// without rounding, and the store rounds once to the element type. Slots hold
-// 2 quads per item. C is at most 2 here (2C quads in flight per thread).
+// without rounding, and the store rounds once to the element type. A slot of
+// the element wire becomes two quad slots (2 * slot, 2 * slot + 1); the host
+// doubles slot_items. C is at most 2 here (2C quads in flight per thread).
 template <class D, int C>
 __global__ void __launch_bounds__(kThreads) k_rd_wide(const KArgs a) {
   pdl_trigger();
@@ -560,31 +608,35 @@ __global__ void __launch_bounds__(kThreads) k_rd_wide(const KArgs a) {
   pdl_wait();
   const unsigned long long ticket = cta_take_ticket(a);
   bool ok = true;
-  for (int64_t base = 0; base < per_chunk; base += stride) {  // same trip count in the whole CTA
+  int64_t rnd = 0;
+  for (int64_t base = 0; base < per_chunk; base += stride, ++rnd) {  // same trip count in the whole CTA
     const int64_t j = base + t0;
     uint4 q[2 * C];
-    int64_t qidx[2 * C];
+    int64_t qslot[2 * C], idx[C];
     bool qval[2 * C];
 #pragma unroll
     for (int k = 0; k < C; ++k) {
-      const int64_t idx = k * per_chunk + j;
-      const bool val = ok && j < per_chunk && idx < a.items;
-      qidx[2 * k] = 2 * idx;
-      qidx[2 * k + 1] = 2 * idx + 1;
+      idx[k] = k * per_chunk + j;
+      const bool val = ok && j < per_chunk && idx[k] < a.items;
+      const int64_t sl = rd_slot(a, k, idx[k], t0, stride);
+      qslot[2 * k] = 2 * sl;
+      qslot[2 * k + 1] = 2 * sl + 1;
       qval[2 * k] = qval[2 * k + 1] = val;
       if (val) {
         Acc<D> x;
-        x.init(load_item_input<D>(a.ptr.in[c.r], idx, a.n));
+        x.init(load_item_input<D>(a.ptr.in[c.r], idx[k], a.n));
         floats_to_quads(x.v, q[2 * k], q[2 * k + 1]);
       }
     }
     if (base == 0) cta_publish_flag(c, ticket);
     if (!ok) continue;
-    ok = rd_exchange<F32T, 2 * C, false>(a, c, q, qidx, qval, 2 * a.items);
+    prefetch_next_round<D, C>(a.ptr.in[c.r], 0, a.items, per_chunk, base, stride, c.b, a.n);
+    ok = rd_exchange<F32T, 2 * C, false>(a, c, q, qslot, qval, a.slot_sets == 1 ? 0 : static_cast<int>(rnd & 1),
+                                         rd_tag(c.flag, rnd));
     if (ok) {
 #pragma unroll
       for (int k = 0; k < C; ++k)
-        if (qval[2 * k]) store_item<D, true>(a.ptr.out[c.r], qidx[2 * k] / 2, a.n, quads_to_item<D>(q[2 * k], q[2 * k + 1]));
+        if (qval[2 * k]) store_item<D, true>(a.ptr.out[c.r], idx[k], a.n, quads_to_item<D>(q[2 * k], q[2 * k + 1]));
     }
   }
 }
@@ -608,26 +660,29 @@ __global__ void __launch_bounds__(kThreads) k_hier_wide(const KArgs a) {
   pdl_wait();
   const unsigned long long ticket = cta_take_ticket(a);
   bool ok = true;
-  for (int64_t base = 0; base < per_chunk; base += stride) {  // same trip count in the whole CTA
+  int64_t rnd = 0;
+  for (int64_t base = 0; base < per_chunk; base += stride, ++rnd) {  // same trip count in the whole CTA
     const int64_t j = base + t0;
     uint4 q[2 * C];
-    int64_t qidx[2 * C];
+    int64_t qslot[2 * C], idx[C];
     bool qval[2 * C];
 #pragma unroll
     for (int k = 0; k < C; ++k) {
-      const int64_t idx = k * per_chunk + j;
-      const bool val = ok && j < per_chunk && idx < len;
-      qidx[2 * k] = 2 * idx;
-      qidx[2 * k + 1] = 2 * idx + 1;
+      idx[k] = k * per_chunk + j;
+      const bool val = ok && j < per_chunk && idx[k] < len;
+      const int64_t sl = rd_slot(a, k, idx[k], t0, stride);
+      qslot[2 * k] = 2 * sl;
+      qslot[2 * k + 1] = 2 * sl + 1;
       qval[2 * k] = qval[2 * k + 1] = val;
       if (val) {
-        const Acc<D> s = reduce_item_acc<D>(a.ptr, g * L, L, lo + idx, a.n);  // not rounded
+        const Acc<D> s = reduce_item_acc<D>(a.ptr, g * L, L, lo + idx[k], a.n);  // not rounded
         floats_to_quads(s.v, q[2 * k], q[2 * k + 1]);
       }
     }
     if (base == 0) cta_publish_flag(c, ticket);
     if (!ok) continue;
-    ok = rd_exchange<F32T, 2 * C, true>(a, c, q, qidx, qval, 2 * piece);
+    ok = rd_exchange<F32T, 2 * C, true>(a, c, q, qslot, qval, a.slot_sets == 1 ? 0 : static_cast<int>(rnd & 1),
+                                        rd_tag(c.flag, rnd));
     if (ok) {
 #pragma unroll
       for (int k = 0; k < C; ++k) {
@@ -635,7 +690,7 @@ __global__ void __launch_bounds__(kThreads) k_hier_wide(const KArgs a) {
         const uint4 v = quads_to_item<D>(q[2 * k], q[2 * k + 1]);
         for (int jj = 0; jj < L; ++jj) {
           const int lp = (l + jj) % L;
-          store_item<D, true>(a.ptr.out[g * L + lp], lo + qidx[2 * k] / 2, a.n, v);
+          store_item<D, true>(a.ptr.out[g * L + lp], lo + idx[k], a.n, v);
         }
       }
     }

@@ -69,9 +69,14 @@ int current_device(int* dev) {
 
 // Allocate (once) the control + signal block and grow the payload slots to at
 // least ll_need bytes. Growing frees the old slots after a device-wide sync.
+// New memory is zeroed with cudaMemset, which runs on the legacy default
+// stream and is not ordered with the caller's stream if that stream was
+// created non-blocking; the device is therefore synchronised after zeroing,
+// so that no kernel on any stream can see the memory before it is zero.
 int ensure_workspace(int dev, size_t ll_need, Workspace** out) {
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& w = g_ws[dev];
+  bool zeroed = false;
   if (!w.ctrl) {
     const size_t words = kCtrlWords + static_cast<size_t>(kPhases) * kSigPhaseWords;
     void* p = nullptr;
@@ -83,6 +88,7 @@ int ensure_workspace(int dev, size_t ll_need, Workspace** out) {
       cudaFree(p);
       return cuda_fail(cudaErrorUnknown);
     }
+    zeroed = true;
     w.ctrl = static_cast<uint32_t*>(p);
     w.sig = w.ctrl + kCtrlWords;
     int sms = 0;
@@ -106,12 +112,20 @@ int ensure_workspace(int dev, size_t ll_need, Workspace** out) {
       cudaFree(p);
       return cuda_fail(cudaErrorUnknown);
     }
+    zeroed = true;
     w.ll = static_cast<uint64_t*>(p);
     w.ll_bytes = bytes;
   }
+  if (zeroed && cudaDeviceSynchronize() != cudaSuccess) return cuda_fail(cudaErrorUnknown);
   *out = &w;
   return VRAR_OK;
 }
+
+// Status and failure info of the allocation-free entry point's control words
+// on device `dev` (defined with that entry point below): reads them into
+// h[kCtrlWords] and clears status and info on the device. *present is false
+// when that entry point has not been set up on the device.
+int noalloc_take_status(int dev, uint32_t* h, bool* present);
 
 // ---- argument checks -------------------------------------------------------------------
 
@@ -167,9 +181,12 @@ bool wide_wire(vrar_algo_t algo, vrar_dtype_t dt) {
          (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER);
 }
 
-// Payload-slot bytes (RD / HIER): P ranks x steps x items-per-slot x 32 bytes,
-// twice that with fp32 partials of 16-bit elements (two quads per item).
-size_t ll_bytes_for(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L) {
+// Payload-slot bytes (RD / HIER) of a call whose grid covers the message in
+// one round: P ranks x steps x items-per-slot x 32 bytes, twice that with fp32
+// partials of 16-bit elements (two quads per item). A call that needs several
+// rounds uses two slot sets of C x (threads per rank) slots instead, which is
+// less than twice this; so twice this bounds every launch of the shape.
+size_t one_round_slot_bytes(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L) {
   const int64_t items = (static_cast<int64_t>(n) + per_item(dt) - 1) / per_item(dt);
   const size_t wide = wide_wire(algo, dt) ? 2 : 1;
   if (algo == VRAR_ALGO_RD) return wide * static_cast<size_t>(P) * ilog2(P) * items * 32;
@@ -178,6 +195,19 @@ size_t ll_bytes_for(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L) {
     return wide * static_cast<size_t>(P) * ilog2(P / L) * piece * 32;
   }
   return 0;
+}
+
+// SM count of a device (cached).
+int device_sms(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  int v = cache[dev].load();
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  cache[dev] = v;
+  return v;
 }
 
 // ---- launch -----------------------------------------------------------------------------
@@ -517,6 +547,64 @@ int rd_chunks_for_dt(vrar_dtype_t dt, vrar_algo_t algo, int C, int64_t work, int
                            : rd_chunks_for<F32T>(algo, C, work, P, dev, sms);
 }
 
+// The launch of a recursive-doubling or hierarchical call and the payload
+// slots it uses (the layout is described with k_rd in kernels.cuh).
+struct PayloadPlan {
+  KernelFn fn = nullptr;
+  int C = 1;                 // payload pieces per thread
+  int B = 1;                 // CTAs per rank
+  int64_t slot_items = 0;    // 32-byte slots per rank, step and slot set
+  int slot_sets = 1;         // 1: one round, slot = item index; 2: slots reused by round parity
+  size_t bytes = 0;          // slot bytes in all: slot_sets * P * steps * slot_items * 32
+};
+
+// C_cfg: the configured chunk count. `fit_one_round` (the allocation-free
+// entry point) takes the smallest chunk count up to the kernels' maximum that
+// covers the message in one round, whatever C_cfg is; if none does, at most 4
+// (at most 1 on the fp32 wire), which keeps its two slot sets below the
+// one-round size.
+int plan_payload(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L, int dev, int sms, int C_cfg,
+                 bool fit_one_round, PayloadPlan* out) {
+  PayloadPlan pl;
+  const bool wide = wide_wire(algo, dt);
+  const int64_t items = (static_cast<int64_t>(n) + per_item(dt) - 1) / per_item(dt);
+  const int64_t piece = algo == VRAR_ALGO_RD ? items : (items + L - 1) / L;  // items one rank exchanges
+  const int steps = algo == VRAR_ALGO_RD ? ilog2(P) : ilog2(P / L);
+  int C = std::min(8, std::max(1, C_cfg));
+  // HIER keeps one payload piece per thread up to 2 MiB per rank and at most
+  // two above: its in-group phases already keep L loads and L stores per
+  // piece in flight, and more pieces cost registers (measured, 4 groups x 8,
+  // both wires; e.g. 226 vs 251 us at 8 MiB, two pieces against four, and
+  // 78 vs 84 us at 2 MiB with fp32 partials, one against two). Above 256 KiB
+  // per rank the element-wire kernel also runs two CTAs per SM (below).
+  if (algo == VRAR_ALGO_HIER) C = n * elem_size(dt) <= kHierOnePieceBytes ? 1 : std::min(C, 2);
+  if (fit_one_round) {
+    const int cmax = wide ? 2 : 8;
+    int pick = 0;
+    for (int c = 1; c <= cmax && !pick; ++c) {
+      KernelFn f = wide ? pick_wide_dt(dt, algo, c) : pick_kernel_dt(dt, algo, c);
+      const int cap = std::max(1, std::min(grid_budget(f, dev, sms), kMaxCtas) / P);
+      if ((piece + c - 1) / c <= static_cast<int64_t>(cap) * kThreads) pick = c;
+    }
+    C = pick ? pick : (wide ? 1 : std::min(C, 4));
+  } else {
+    C = wide ? wide_chunks_for(dt, algo, C, piece, P, dev, sms) : rd_chunks_for_dt(dt, algo, C, piece, P, dev, sms);
+  }
+  pl.C = C;
+  pl.fn = wide ? pick_wide_dt(dt, algo, C) : pick_kernel_dt(dt, algo, C);
+  if (algo == VRAR_ALGO_HIER && !wide && n * elem_size(dt) > kHierOneCtaBytes) pl.fn = hier_two_per_sm_dt(dt, C);
+  if (!pl.fn) return VRAR_EINVAL;
+  const int64_t per_chunk = (piece + C - 1) / C;
+  pl.B = blocks_per_rank(per_chunk, P, grid_budget(pl.fn, dev, sms));
+  const int64_t stride = static_cast<int64_t>(pl.B) * kThreads;
+  const int64_t rounds = (per_chunk + stride - 1) / stride;
+  pl.slot_sets = rounds > 1 ? 2 : 1;
+  pl.slot_items = (rounds > 1 ? static_cast<int64_t>(C) * stride : piece) * (wide ? 2 : 1);
+  pl.bytes = static_cast<size_t>(pl.slot_sets) * P * steps * pl.slot_items * 32;
+  *out = pl;
+  return VRAR_OK;
+}
+
 const char* algo_name(int a) {
   switch (a) {
     case VRAR_ALGO_ONESHOT: return "oneshot";
@@ -569,26 +657,16 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
 
   int dev = 0;
   if ((rc = current_device(&dev)) != VRAR_OK) return rc;
+  const int sms = device_sms(dev);
+  if (sms < 1) return VRAR_ECUDA;
+  const bool payload = algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER;
+  PayloadPlan plan;
+  if (payload && (rc = plan_payload(algo, P, n, dtype, L, dev, sms, g_set.rd_chunks.load(), false, &plan)) != VRAR_OK)
+    return rc;
   Workspace* ws = nullptr;
-  if ((rc = ensure_workspace(dev, ll_bytes_for(algo, P, n, dtype, L), &ws)) != VRAR_OK) return rc;
-
-  int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
-  const bool wide = wide_wire(algo, dtype);
-  // HIER keeps one payload piece per thread up to 2 MiB per rank and at most
-  // two above: its in-group phases already keep L loads and L stores per
-  // piece in flight, and more pieces cost registers (measured, 4 groups x 8,
-  // both wires; e.g. 226 vs 251 us at 8 MiB, two pieces against four, and
-  // 78 vs 84 us at 2 MiB with fp32 partials, one against two). Above 256 KiB
-  // per rank the element-wire kernel also runs two CTAs per SM (below).
-  if (algo == VRAR_ALGO_HIER) C = n * elem_size(dtype) <= kHierOnePieceBytes ? 1 : std::min(C, 2);
-  if (algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER) {
-    const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
-    const int64_t work = algo == VRAR_ALGO_RD ? items : (items + L - 1) / L;
-    C = wide ? wide_chunks_for(dtype, algo, C, work, P, dev, ws->sms)
-             : rd_chunks_for_dt(dtype, algo, C, work, P, dev, ws->sms);
-  }
-  KernelFn fn = wide ? pick_wide_dt(dtype, algo, C) : pick_kernel_dt(dtype, algo, C);
-  if (algo == VRAR_ALGO_HIER && !wide && n * elem_size(dtype) > kHierOneCtaBytes) fn = hier_two_per_sm_dt(dtype, C);
+  if ((rc = ensure_workspace(dev, payload ? plan.bytes : 0, &ws)) != VRAR_OK) return rc;
+  const int C = payload ? plan.C : 1;
+  KernelFn fn = payload ? plan.fn : pick_kernel_dt(dtype, algo, 1);
   if (!fn) return VRAR_EINVAL;
 
   KArgs a;
@@ -608,34 +686,31 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   a.ctrl = ws->ctrl;
   a.sig = ws->sig;
   a.ll = ws->ll;
+  a.slot_items = plan.slot_items;
+  a.slot_sets = plan.slot_sets;
   a.stats = g_set.spin_stats.load() ? reinterpret_cast<unsigned long long*>(ws->ctrl + kStats) : nullptr;
+  if (payload) {
+    a.steps = algo == VRAR_ALGO_RD ? ilog2(P) : ilog2(P / L);
+    a.B = plan.B;
+    return launch(plan.fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
+  }
 
   int64_t work = a.items;  // items one rank handles in its main loop
   switch (algo) {
     case VRAR_ALGO_ONESHOT: work = a.items; break;
     case VRAR_ALGO_TWOSTAGE:
     case VRAR_ALGO_TWOSTAGE_WRITE: work = (a.items + P - 1) / P; break;
-    case VRAR_ALGO_RD:
-      a.steps = ilog2(P);
-      work = (a.items + C - 1) / C;
-      break;
-    case VRAR_ALGO_HIER: {
-      a.steps = ilog2(P / L);
-      const int64_t piece = (a.items + L - 1) / L;
-      work = (piece + C - 1) / C;
-      break;
-    }
     default: break;
   }
   const int wk = algo == VRAR_ALGO_TWOSTAGE_WRITE ? write_kernel_for(P, n * elem_size(dtype)) : kWritePlain;
   if (wk == kWriteAsync) {
     const int cap_budget = g_set.max_ctas.load();
-    const bool deep = cap_budget > 0 && cap_budget <= ws->sms;
+    const bool deep = cap_budget > 0 && cap_budget <= sms;
     const int S = async_stages(P, n * elem_size(dtype), deep);
     KernelFn af = async_kernel_dt(dtype, S);
     const int64_t tiles = std::max<int64_t>(1, (work + kAsyncTileItems - 1) / kAsyncTileItems);
     const size_t smem = static_cast<size_t>(S) * P * kAsyncTileItems * 16;
-    const int resident = grid_budget(af, dev, ws->sms, kAsyncTileItems, smem);
+    const int resident = grid_budget(af, dev, sms, kAsyncTileItems, smem);
     if (resident < 1) return VRAR_ECUDA;
     a.B = static_cast<int>(std::min<int64_t>(tiles, std::max(1, std::min(resident, kMaxCtas) / P)));
     return launch(af, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), kAsyncTileItems, smem);
@@ -646,13 +721,13 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     // far more bytes in flight to draw its share of memory bandwidth: 128-item
     // tiles and up to 192 KiB of stages.
     const int cap_budget = g_set.max_ctas.load();
-    const bool deep = cap_budget > 0 && cap_budget <= ws->sms;
+    const bool deep = cap_budget > 0 && cap_budget <= sms;
     const int ti = deep ? 128 : kWriteTileItems;
     KernelFn sf = staged_kernel_dt(dtype, ti);
     const int64_t tiles = std::max<int64_t>(1, (work + ti - 1) / ti);
     const int S = std::max(2, std::min(deep ? kMaxStages : 6, ((deep ? 192 : 96) * 1024) / (P * ti * 16)));
     const size_t smem = kStagedHeader + static_cast<size_t>(S) * P * ti * 16;
-    const int resident = grid_budget(sf, dev, ws->sms, 32 + ti, smem);
+    const int resident = grid_budget(sf, dev, sms, 32 + ti, smem);
     const int B = static_cast<int>(std::min<int64_t>(tiles, std::max(1, std::min(resident, kMaxCtas) / P)));
     if (resident < 1) return VRAR_ECUDA;
     a.stages = S;
@@ -668,7 +743,7 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     fn = pull_dt(dtype);
     threads = kPullThreads;
   }
-  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, ws->sms, threads), threads);
+  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, sms, threads), threads);
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), threads);
 }
 
@@ -681,6 +756,8 @@ int vrar_reduce_scatter(const void* const rank_in[], void* const rank_out[], int
   if (n == 0) return VRAR_OK;
   int dev = 0;
   if ((rc = current_device(&dev)) != VRAR_OK) return rc;
+  const int sms = device_sms(dev);
+  if (sms < 1) return VRAR_ECUDA;
   Workspace* ws = nullptr;
   if ((rc = ensure_workspace(dev, 0, &ws)) != VRAR_OK) return rc;
   KernelFn fn = dtype == VRAR_BF16   ? k_reduce_scatter<Bf16T>
@@ -704,17 +781,17 @@ int vrar_reduce_scatter(const void* const rank_in[], void* const rank_out[], int
     const int64_t mi = m / per_item(dtype);
     a.items = mi * P;
     const int cap_budget = g_set.max_ctas.load();
-    const int S = async_stages(P, n * elem_size(dtype), cap_budget > 0 && cap_budget <= ws->sms);
+    const int S = async_stages(P, n * elem_size(dtype), cap_budget > 0 && cap_budget <= sms);
     KernelFn af = async_rs_kernel_dt(dtype, S);
     const int64_t tiles = std::max<int64_t>(1, (mi + kAsyncTileItems - 1) / kAsyncTileItems);
     const size_t smem = static_cast<size_t>(S) * P * kAsyncTileItems * 16;
-    const int resident = grid_budget(af, dev, ws->sms, kAsyncTileItems, smem);
+    const int resident = grid_budget(af, dev, sms, kAsyncTileItems, smem);
     if (resident < 1) return VRAR_ECUDA;
     a.B = static_cast<int>(std::min<int64_t>(tiles, std::max(1, std::min(resident, kMaxCtas) / P)));
     return launch(af, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), kAsyncTileItems, smem);
   }
   const int64_t work = (m % per_item(dtype) == 0) ? m / per_item(dtype) : m;
-  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, ws->sms));
+  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, sms));
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -727,6 +804,8 @@ int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, 
   if (n == 0) return VRAR_OK;
   int dev = 0;
   if ((rc = current_device(&dev)) != VRAR_OK) return rc;
+  const int sms = device_sms(dev);
+  if (sms < 1) return VRAR_ECUDA;
   Workspace* ws = nullptr;
   if ((rc = ensure_workspace(dev, 0, &ws)) != VRAR_OK) return rc;
   KernelFn fn = dtype == VRAR_BF16   ? k_all_gather<Bf16T>
@@ -742,7 +821,7 @@ int vrar_all_gather(const void* const rank_in[], void* const rank_out[], int P, 
   a.P = P;
   const int64_t m = a.n / P;
   const int64_t work = (m % per_item(dtype) == 0) ? m / per_item(dtype) : m;
-  const int budget = grid_budget(fn, dev, ws->sms);
+  const int budget = grid_budget(fn, dev, sms);
   a.B = blocks_per_rank(work, P, budget);
   // Destination groups: fill the resident grid when the slices are short.
   a.chunks = std::max(1, std::min(P, budget / (a.B * P)));
@@ -807,19 +886,36 @@ int vrar_query_status(vrar_stream_t stream, uint32_t info[4]) {
   int rc = current_device(&dev);
   if (rc != VRAR_OK) return rc;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
-  std::lock_guard<std::mutex> lock(g_mu);
-  Workspace& w = g_ws[dev];
   if (info) std::memset(info, 0, 4 * sizeof(uint32_t));
-  if (!w.ctrl) return VRAR_OK;
+  uint32_t status = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    Workspace& w = g_ws[dev];
+    if (w.ctrl) {
+      uint32_t h[kCtrlWords];
+      if (cudaMemcpy(h, w.ctrl, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+      if (h[kStatus] != 0) {
+        status = h[kStatus];
+        if (info) std::memcpy(info, h + kInfo, 4 * sizeof(uint32_t));
+        const uint32_t zero[5] = {0, 0, 0, 0, 0};
+        if (cudaMemcpy(w.ctrl + kStatus, zero, sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
+            cudaMemcpy(w.ctrl + kInfo, zero, 4 * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess)
+          return cuda_fail(cudaErrorUnknown);
+      }
+    }
+  }
+  // The allocation-free entry point keeps its own control words in its fixed
+  // array; a failure there is reported here too (after the workspace's, whose
+  // info wins if both failed), and cleared.
   uint32_t h[kCtrlWords];
-  if (cudaMemcpy(h, w.ctrl, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
-  if (h[kStatus] == 0) return VRAR_OK;
-  if (info) std::memcpy(info, h + kInfo, 4 * sizeof(uint32_t));
-  const uint32_t zero[5] = {0, 0, 0, 0, 0};
-  if (cudaMemcpy(w.ctrl + kStatus, zero, sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(w.ctrl + kInfo, zero, 4 * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess)
-    return cuda_fail(cudaErrorUnknown);
-  return h[kStatus] == kErrTimeout ? VRAR_ETIMEDOUT : VRAR_ECUDA;
+  bool present = false;
+  if ((rc = noalloc_take_status(dev, h, &present)) != VRAR_OK) return rc;
+  if (present && h[kStatus] != 0 && status == 0) {
+    status = h[kStatus];
+    if (info) std::memcpy(info, h + kInfo, 4 * sizeof(uint32_t));
+  }
+  if (status == 0) return VRAR_OK;
+  return status == kErrTimeout ? VRAR_ETIMEDOUT : VRAR_ECUDA;
 }
 
 int vrar_reserve(size_t bytes) {
@@ -835,7 +931,16 @@ size_t vrar_workspace_bytes(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t alg
   if (algo == VRAR_ALGO_AUTO) algo = static_cast<vrar_algo_t>(select_algo(P, n, dtype));
   const int L = g_set.group_size.load();
   if (check_shape(algo, P, L) != VRAR_OK) return 0;
-  return ll_bytes_for(algo, P, n, dtype, L);
+  if (algo != VRAR_ALGO_RD && algo != VRAR_ALGO_HIER) return 0;
+  int dev = 0;
+  int sms = 0;
+  if (n > 0 && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices && (sms = device_sms(dev)) > 0) {
+    PayloadPlan plan;
+    if (plan_payload(algo, P, n, dtype, L, dev, sms, g_set.rd_chunks.load(), false, &plan) == VRAR_OK)
+      return plan.bytes;
+  }
+  cudaGetLastError();
+  return 2 * one_round_slot_bytes(algo, P, n, dtype, L);  // no usable device: the bound for any grid
 }
 
 int vrar_reset(void) {
@@ -936,16 +1041,19 @@ std::mutex g_noalloc_mu;
 NoAllocDevice g_noalloc[kMaxDevices];
 
 // Once per device, with that device current: look up the array's device
-// address, zero it (so no payload word or ticket starts with a value a call
-// could take for its own), and read the SM count for grid sizing.
-int noalloc_setup(int dev, NoAllocDevice** out) {
+// address and read the SM count for grid sizing. The array is zero when the
+// library's module is loaded; the set-up zeroes it once more on the caller's
+// stream (cudaMemsetAsync, ordered before the call's kernel on that stream, so
+// it cannot race with it whatever the stream's flags), so that no payload word
+// or ticket starts with a value a call could take for its own.
+int noalloc_setup(int dev, cudaStream_t stream, NoAllocDevice** out) {
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   NoAllocDevice& d = g_noalloc[dev];
   if (!d.base) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) return cuda_fail(e);
-    if (cudaMemset(p, 0, kNoAllocBytes) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
+    if (cudaMemsetAsync(p, 0, kNoAllocBytes, stream) != cudaSuccess) return cuda_fail(cudaErrorUnknown);
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return cuda_fail(cudaErrorUnknown);
@@ -953,6 +1061,24 @@ int noalloc_setup(int dev, NoAllocDevice** out) {
     d.base = static_cast<unsigned char*>(p);
   }
   *out = &d;
+  return VRAR_OK;
+}
+
+// The status half of vrar_query_status for the fixed array (declared above).
+// The caller has synchronised the stream it asks about.
+int noalloc_take_status(int dev, uint32_t* h, bool* present) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  *present = g_noalloc[dev].base != nullptr;
+  if (!*present) return VRAR_OK;
+  uint32_t* ctrl = reinterpret_cast<uint32_t*>(g_noalloc[dev].base);
+  if (cudaMemcpy(h, ctrl, kCtrlWords * sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_fail(cudaErrorUnknown);
+  if (h[kStatus] != 0) {
+    const uint32_t zero[5] = {0, 0, 0, 0, 0};
+    if (cudaMemcpy(ctrl + kStatus, zero, sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(ctrl + kInfo, zero, 4 * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess)
+      return cuda_fail(cudaErrorUnknown);
+  }
   return VRAR_OK;
 }
 
@@ -965,20 +1091,21 @@ extern "C" int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* cons
   if (rc != VRAR_OK) return rc;
   if ((rc = check_shape(VRAR_ALGO_RD, P, 1)) != VRAR_OK) return rc;
   const int64_t items = (static_cast<int64_t>(n) + per_item(dtype) - 1) / per_item(dtype);
-  const size_t slots = ll_bytes_for(VRAR_ALGO_RD, P, n, dtype, 1);
-  if (static_cast<size_t>(items) > kNoAllocBytes || slots > kNoAllocBytes - kNoAllocCtrlBytes) return VRAR_ETOOBIG;
+  // The documented limit: the one-round slot size must fit beside the control
+  // words. The launch planned below never needs more than that.
+  if (static_cast<size_t>(items) > kNoAllocBytes ||
+      one_round_slot_bytes(VRAR_ALGO_RD, P, n, dtype, 1) > kNoAllocBytes - kNoAllocCtrlBytes)
+    return VRAR_ETOOBIG;
   if (n == 0) return VRAR_OK;
 
   int dev = 0;
   if ((rc = current_device(&dev)) != VRAR_OK) return rc;
   NoAllocDevice* d = nullptr;
-  if ((rc = noalloc_setup(dev, &d)) != VRAR_OK) return rc;
-
-  int C = std::min(8, std::max(1, g_set.rd_chunks.load()));
-  const bool wide = wide_wire(VRAR_ALGO_RD, dtype);
-  C = wide ? wide_chunks_for(dtype, VRAR_ALGO_RD, C, items, P, dev, d->sms)
-           : rd_chunks_for_dt(dtype, VRAR_ALGO_RD, C, items, P, dev, d->sms);
-  KernelFn fn = wide ? pick_wide_dt(dtype, VRAR_ALGO_RD, C) : pick_kernel_dt(dtype, VRAR_ALGO_RD, C);
+  if ((rc = noalloc_setup(dev, reinterpret_cast<cudaStream_t>(stream), &d)) != VRAR_OK) return rc;
+  PayloadPlan plan;
+  if ((rc = plan_payload(VRAR_ALGO_RD, P, n, dtype, 1, dev, d->sms, g_set.rd_chunks.load(), true, &plan)) != VRAR_OK)
+    return rc;
+  if (plan.bytes > kNoAllocBytes - kNoAllocCtrlBytes) return VRAR_ETOOBIG;
   KArgs a;
   std::memset(&a, 0, sizeof(a));
   for (int p = 0; p < P; ++p) {
@@ -990,12 +1117,14 @@ extern "C" int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* cons
   a.P = P;
   a.L = 1;
   a.steps = ilog2(P);
-  a.chunks = C;
-  a.fault_mask = 0;
+  a.chunks = plan.C;
+  a.fault_mask = g_set.fault_mask.load();
   a.timeout_ns = g_set.timeout_ns.load();
   a.ctrl = reinterpret_cast<uint32_t*>(d->base);
   a.sig = nullptr;  // recursive doubling uses no barrier rows
   a.ll = reinterpret_cast<uint64_t*>(d->base + kNoAllocCtrlBytes);
-  a.B = blocks_per_rank((a.items + C - 1) / C, P, grid_budget(fn, dev, d->sms));
-  return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
+  a.slot_items = plan.slot_items;
+  a.slot_sets = plan.slot_sets;
+  a.B = plan.B;
+  return launch(plan.fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
 }

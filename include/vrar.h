@@ -220,12 +220,15 @@ VRAR_API int vrar_set_spin_timeout_ns(uint64_t ns);
 VRAR_API uint64_t vrar_get_spin_timeout_ns(void);
 
 /*
- * Wait for `stream`, then return and clear the device status word of the
+ * Wait for `stream`, then return and clear the device status words of the
  * current device: VRAR_OK, or VRAR_ETIMEDOUT if any wait of any call since
- * the last query ran out of time. If info is not NULL it receives details of
- * the first failure: info[0] = call sequence number, info[1] = phase
- * (1 start, 2 mid, 3 end, 4 payload, 5 shared-memory stage of the bulk-copy
- * write kernel), info[2] = waiting rank, info[3] = block.
+ * the last query ran out of time. This covers the calls that use the
+ * library's workspace and those of vrar_allreduce_rd_noalloc, whose status
+ * words live in its fixed array; both are cleared. If info is not NULL it
+ * receives details of the first failure (the workspace's, if both failed):
+ * info[0] = call sequence number, info[1] = phase (1 start, 2 mid, 3 end,
+ * 4 payload, 5 shared-memory stage of the bulk-copy write kernel),
+ * info[2] = waiting rank, info[3] = block. Allocates nothing.
  */
 VRAR_API int vrar_query_status(vrar_stream_t stream, uint32_t info[4]);
 
@@ -279,16 +282,19 @@ VRAR_API int vrar_debug_set_fault_mask(uint32_t mask);
  *    e = 8 for bf16 / fp16, 4 for fp32 (P = 8, bf16: n <= 174,760). Larger
  *    requests return VRAR_ETOOBIG before anything is queued.
  *  - The first call on a device sets that device up: it looks up the array's
- *    device address (cudaGetSymbolAddress) and zeroes it, which waits for the
- *    device. Make that first call before any stream capture.
+ *    device address (cudaGetSymbolAddress) and queues the array's zeroing
+ *    (cudaMemsetAsync) on `stream`, ahead of the call's kernel. Make that
+ *    first call before any stream capture.
  *  - All calls on a device share the one array, and it keeps the last call's
  *    contents; nothing has to be cleared between calls, because every word a
  *    call waits for carries that call's sequence number. Calls that overlap on
  *    the GPU (on different streams, or from several host threads) race on the
  *    array and give wrong results: keep them ordered on one stream.
- *  - Device waits are bounded as in every other call, but a wait that runs out
- *    of time is not reported anywhere the host can read (vrar_query_status
- *    covers the allocated workspace only).
+ *  - Device waits are bounded as in every other call (vrar_set_spin_timeout_ns)
+ *    and honour vrar_debug_set_fault_mask. A wait that runs out of time
+ *    records VRAR_ETIMEDOUT in the array's status word, and the outputs of the
+ *    items whose waits gave up are left unwritten; vrar_query_status reports
+ *    and clears it. Spin statistics are not collected on this path.
  */
 #define VRAR_NOALLOC_SCRATCH_BYTES (16u << 20)
 VRAR_API int vrar_allreduce_rd_noalloc(const void* const rank_in[], void* const rank_out[], int P, size_t n,

@@ -12,20 +12,30 @@
 //  * one 64-bit ticket per device: every CTA of a call adds 1; the CTA that
 //    brings the low half to the grid size also adds 2^32 - grid, so the high
 //    half counts calls and the low half returns to 0. A CTA's flag for the
-//    call is (high half before its add) + 1.
+//    call is (high half before its add) mod (2^31 - 1) + 1: never 0, below 2^31.
 //  * a barrier: CTA (r, b) stores the flag into word [(p*B + b)*32 + r] of the
 //    phase's array for every rank p (release), then waits until word
 //    [(r*B + b)*32 + p] equals the flag for every p (acquire). Words are never
 //    cleared; equality with a flag that only grows rejects every stale word.
-//  * recursive doubling: at step s rank r stores {data | flag << 32} into
-//    the step-s slot of partner r XOR 2^s and polls its own step-s slot until
-//    the high half equals the flag, then adds.
+//  * recursive doubling in rounds: a rank's items are cut into C chunks and
+//    covered by S = B * T thread positions per round (T per CTA); in round t
+//    position t0 holds item k*per_chunk + t*S + t0 of every chunk k. At step s
+//    rank r stores {data | tag << 32} into the step-s slot of partner
+//    r XOR 2^s and polls its own step-s slot until the high half equals the
+//    tag, then adds. With one round the slot of an item is its index; with
+//    several, piece k of position t0 uses slot k*S + t0 of slot set (t & 1),
+//    and the tag of round t is the flag with bit 31 set to bit 1 of t. A slot
+//    is rewritten two rounds later only after its reader has read it (the
+//    writer needs the reader's next-round word first), and the lap bit keeps
+//    a word from two rounds back from passing for the current one.
 //  * every wait is bounded; the first CTA to give up records a status and the
 //    call's flag as the failed epoch, and every other wait of that call stops
 //    as soon as it sees the epoch.
 //
-// Checks: thousands of back-to-back calls whose shape (P, B, items) changes
-// from call to call, each with exact integer sums on every rank from both the
+// Checks: thousands of back-to-back calls whose shape (P, B, items, C)
+// changes from call to call, many of them several rounds long, with one rank
+// per call held back (before its first poll, and before its sends two rounds
+// later), each with exact integer sums on every rank from both the
 // recursive doubling and the pull 2-stage (a stale or early word, or a read
 // that the mid barrier did not order after its write, would change them; one
 // rank per call writes its 2-stage slice late, and under ThreadSanitizer the
@@ -43,7 +53,8 @@
 // Planted mistakes for the tests (0 = the protocol as specified): 1 the
 // payload poll ignores the sequence number; 2 the ticket's last arriver does
 // not return the low half to 0 (every call then has the same flag); 3 a
-// barrier posts into the waiter's own words instead of the peers'.
+// barrier posts into the waiter's own words instead of the peers'; 4 the
+// rounds of a call share one slot set; 5 round tags carry no lap bit.
 #ifndef MODEL_MUTANT
 #define MODEL_MUTANT 0
 #endif
@@ -55,6 +66,7 @@ constexpr int kMaxB = 4;
 constexpr int kPhases = 3;  // start, mid, end
 constexpr int kMaxSteps = 5;
 constexpr int kMaxItems = 64;  // items per rank
+constexpr int kT = 2;          // thread positions per CTA in the recursive doubling
 // Waits are bounded by time, as on the device (where the limit is 2 s by
 // default and read from %globaltimer); a poll count would give up on a peer
 // thread that the OS has simply not scheduled yet.
@@ -66,14 +78,14 @@ struct Device {
   std::atomic<uint32_t> fail_epoch{0};
   std::vector<std::atomic<uint32_t>> sig;
   std::vector<std::atomic<uint64_t>> ll;
-  Device() : sig(kPhases * kMaxB * kMaxP * kMaxP), ll(kMaxP * kMaxSteps * kMaxItems) {
+  Device() : sig(kPhases * kMaxB * kMaxP * kMaxP), ll(2 * kMaxP * kMaxSteps * kMaxItems) {
     for (auto& w : sig) w.store(0);
     for (auto& w : ll) w.store(0);
   }
 };
 
 struct Call {
-  int P, B, items, steps;
+  int P, B, items, steps, C;
   int muted;  // rank that never posts or sends, -1 for none
   std::vector<int32_t> in, out;  // [P][items]; out: recursive doubling's result
   std::vector<int32_t> pull;     // [P][items]: the pull 2-stage's result (plain, not atomic)
@@ -84,7 +96,7 @@ uint32_t take_flag(Device& d, int grid) {
   const uint64_t old = d.ticket.fetch_add(1, std::memory_order_acq_rel);
   if (MODEL_MUTANT != 2 && static_cast<uint32_t>(old) == static_cast<uint32_t>(grid - 1))
     d.ticket.fetch_add((uint64_t{1} << 32) - static_cast<uint64_t>(grid), std::memory_order_acq_rel);
-  return static_cast<uint32_t>(old >> 32) + 1;
+  return static_cast<uint32_t>(old >> 32) % 0x7FFFFFFFu + 1u;
 }
 
 // Bounded wait for `word == flag`; false once the limit passes or the call's
@@ -117,29 +129,60 @@ bool barrier(Device& d, const Call& c, int phase, int r, int b, uint32_t flag) {
   return true;
 }
 
-// CTA (r, b): start barrier; recursive doubling over its items (b, b+B, ...);
-// the pull 2-stage on the same items (phase 1: rank r sums its slice into
-// pull[r]; mid barrier; phase 2: it copies every other slice s out of
-// pull[s]); store; end barrier.
+// CTA (r, b): start barrier; recursive doubling over its thread positions
+// b*kT .. b*kT + kT - 1, round by round; the pull 2-stage on the items b, b+B,
+// ... (phase 1: rank r sums its slice into pull[r]; mid barrier; phase 2: it
+// copies every other slice s out of pull[s]); store; end barrier.
 void cta(Device& d, Call& c, int r, int b) {
   const uint32_t flag = take_flag(d, c.P * c.B);
   if (!barrier(d, c, 0, r, b, flag)) return;
-  std::vector<int32_t> v;
-  for (int i = b; i < c.items; i += c.B) v.push_back(c.in[r * c.items + i]);
-  for (int s = 0; s < c.steps; ++s) {
-    const int q = r ^ (1 << s);
-    size_t k = 0;
-    for (int i = b; i < c.items; i += c.B, ++k)
-      if (r != c.muted)
-        d.ll[(static_cast<size_t>(q) * kMaxSteps + s) * kMaxItems + i].store(
-            (static_cast<uint64_t>(flag) << 32) | static_cast<uint32_t>(v[k]), std::memory_order_release);
-    k = 0;
-    for (int i = b; i < c.items; i += c.B, ++k) {
-      auto& w = d.ll[(static_cast<size_t>(r) * kMaxSteps + s) * kMaxItems + i];
-      if (!wait_for(d, w, flag, [&](uint64_t x) { return MODEL_MUTANT == 1 || static_cast<uint32_t>(x >> 32) == flag; }))
-        return;
-      v[k] += static_cast<int32_t>(static_cast<uint32_t>(w.load(std::memory_order_acquire)));
+  const int S = c.B * kT;
+  const int per_chunk = (c.items + c.C - 1) / c.C;
+  const int rounds = (per_chunk + S - 1) / S;
+  const bool reuse = rounds > 1;
+  for (int rnd = 0, base = 0; base < per_chunk; base += S, ++rnd) {
+    const int set = (reuse && MODEL_MUTANT != 4) ? (rnd & 1) : 0;
+    const uint32_t tag = MODEL_MUTANT == 5 ? flag : flag | (static_cast<uint32_t>((rnd >> 1) & 1) << 31);
+    int idx[kT][8], slot[kT][8];
+    bool val[kT][8];
+    int32_t v[kT][8];
+    for (int u = 0; u < kT; ++u) {
+      const int t0 = b * kT + u, j = base + t0;
+      for (int k = 0; k < c.C; ++k) {
+        idx[u][k] = k * per_chunk + j;
+        slot[u][k] = reuse ? k * S + t0 : idx[u][k];
+        val[u][k] = j < per_chunk && idx[u][k] < c.items;
+        v[u][k] = val[u][k] ? c.in[r * c.items + idx[u][k]] : 0;
+      }
     }
+    for (int s = 0; s < c.steps; ++s) {
+      const int q = r ^ (1 << s);
+      std::atomic<uint64_t>* dst = &d.ll[((static_cast<size_t>(set) * kMaxP + q) * kMaxSteps + s) * kMaxItems];
+      std::atomic<uint64_t>* src = &d.ll[((static_cast<size_t>(set) * kMaxP + r) * kMaxSteps + s) * kMaxItems];
+      if (r == c.late && rnd == 2 && s == 0) std::this_thread::sleep_for(std::chrono::microseconds(200));
+      if (r != c.muted)
+        for (int u = 0; u < kT; ++u)
+          for (int k = 0; k < c.C; ++k)
+            if (val[u][k])
+              dst[slot[u][k]].store((static_cast<uint64_t>(tag) << 32) | static_cast<uint32_t>(v[u][k]),
+                                    std::memory_order_release);
+      if (r == c.late && rnd == 0 && s == 0) std::this_thread::sleep_for(std::chrono::microseconds(200));
+      for (int u = 0; u < kT; ++u)
+        for (int k = 0; k < c.C; ++k) {
+          if (!val[u][k]) continue;
+          auto& w = src[slot[u][k]];
+          uint64_t got = 0;
+          if (!wait_for(d, w, flag, [&](uint64_t x) {
+                got = x;
+                return MODEL_MUTANT == 1 || static_cast<uint32_t>(x >> 32) == tag;
+              }))
+            return;
+          v[u][k] += static_cast<int32_t>(static_cast<uint32_t>(got));
+        }
+    }
+    for (int u = 0; u < kT; ++u)
+      for (int k = 0; k < c.C; ++k)
+        if (val[u][k]) c.out[r * c.items + idx[u][k]] = v[u][k];
   }
   const int piece = (c.items + c.P - 1) / c.P;
   auto slice_lo = [&](int s) { return s * piece < c.items ? s * piece : c.items; };
@@ -156,8 +199,6 @@ void cta(Device& d, Call& c, int r, int b) {
     for (int i = slice_lo(s); i < slice_lo(s + 1); ++i)
       if (i % c.B == b) c.pull[r * c.items + i] = c.pull[s * c.items + i];
   }
-  size_t k = 0;
-  for (int i = b; i < c.items; i += c.B, ++k) c.out[r * c.items + i] = v[k];
   barrier(d, c, 2, r, b, flag);
 }
 
@@ -168,8 +209,8 @@ void run(Device& d, Call& c) {
   for (auto& t : ts) t.join();  // the next call starts after this one: stream order
 }
 
-Call make_call(int k, int P, int B, int items, int muted) {
-  Call c{P, B, items, 0, muted, std::vector<int32_t>(P * items), std::vector<int32_t>(P * items, 0),
+Call make_call(int k, int P, int B, int items, int C, int muted) {
+  Call c{P, B, items, 0, C, muted, std::vector<int32_t>(P * items), std::vector<int32_t>(P * items, 0),
          std::vector<int32_t>(P * items, 0), k % P};
   while ((1 << c.steps) < P) ++c.steps;
   for (int p = 0; p < P; ++p)
@@ -192,20 +233,23 @@ bool exact(const Call& c) {
 int main(int argc, char** argv) {
   const int calls = argc > 1 ? std::atoi(argv[1]) : 3000;
   Device d;
-  const int shapes[][3] = {{2, 1, 5}, {4, 2, 17}, {8, 1, 33}, {8, 4, 64}, {16, 2, 9}, {32, 1, 3}, {4, 4, 1}};
+  // {P, B, items, C}: one-round and many-round calls (up to 32 rounds).
+  constexpr int kShapes = 10;
+  const int shapes[kShapes][4] = {{2, 1, 5, 1},  {4, 2, 17, 2}, {8, 1, 33, 1}, {8, 4, 64, 2}, {16, 2, 9, 1},
+                                  {32, 1, 3, 1}, {4, 4, 1, 3},  {2, 1, 64, 1}, {4, 1, 60, 3}, {8, 2, 64, 3}};
   for (int k = 0; k < calls; ++k) {
-    const auto& sh = shapes[k % 7];
-    Call c = make_call(k, sh[0], sh[1], sh[2], -1);
+    const auto& sh = shapes[k % kShapes];
+    Call c = make_call(k, sh[0], sh[1], sh[2], sh[3], -1);
     run(d, c);
     if (d.status.load() != 0 || !exact(c)) {
-      std::fprintf(stderr, "call %d (P=%d B=%d items=%d): status %u, exact %d\n", k, c.P, c.B, c.items,
+      std::fprintf(stderr, "call %d (P=%d B=%d items=%d C=%d): status %u, exact %d\n", k, c.P, c.B, c.items, c.C,
                    d.status.load(), exact(c) ? 1 : 0);
       return 1;
     }
   }
   // A rank that never posts or sends: every wait of the call gives up, the
   // status is recorded, every thread returns.
-  Call bad = make_call(calls, 8, 2, 20, 3);
+  Call bad = make_call(calls, 8, 2, 20, 2, 3);
   run(d, bad);
   if (d.status.load() != 1) {
     std::fprintf(stderr, "missing rank: status %u\n", d.status.load());
@@ -215,8 +259,8 @@ int main(int argc, char** argv) {
   // Later calls are correct again: their flags are new, so no word written in
   // the failed call (or before it) can match.
   for (int k = calls + 1; k < calls + 50; ++k) {
-    const auto& sh = shapes[k % 7];
-    Call c = make_call(k, sh[0], sh[1], sh[2], -1);
+    const auto& sh = shapes[k % kShapes];
+    Call c = make_call(k, sh[0], sh[1], sh[2], sh[3], -1);
     run(d, c);
     if (d.status.load() != 0 || !exact(c)) {
       std::fprintf(stderr, "after the failure, call %d: status %u, exact %d\n", k, d.status.load(), exact(c) ? 1 : 0);

@@ -189,9 +189,11 @@ def test_payload_wire_setting():
     try:
         assert vrar.get_payload_wire() == "fp32"
         # fp32 partials of bf16: twice the slot bytes; fp32 elements unchanged; one-shot needs none
-        assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 2 * 8 * 3 * 131072 * 32
-        assert vrar.workspace_bytes(8, 1 << 20, torch.float32, "rd") == 8 * 3 * 262144 * 32
-        assert vrar.workspace_bytes(32, 1 << 20, torch.float16, "hier") == 2 * 32 * 2 * 16384 * 32
+        # (no device here: the bound for any grid, twice the one-round size)
+        if not torch.cuda.is_available():
+            assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 2 * 2 * 8 * 3 * 131072 * 32
+            assert vrar.workspace_bytes(8, 1 << 20, torch.float32, "rd") == 2 * 8 * 3 * 262144 * 32
+            assert vrar.workspace_bytes(32, 1 << 20, torch.float16, "hier") == 2 * 2 * 32 * 2 * 16384 * 32
         assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "oneshot") == 0
         # the allocation-free entry point's limit halves for bf16 with fp32 partials
         f = L.vrar_allreduce_rd_noalloc
@@ -200,10 +202,17 @@ def test_payload_wire_setting():
         vrar.set_payload_wire("element")
 
 
-def test_workspace_bytes():
-    # RD at P=8 on 2 MiB of bf16 per rank: 8 ranks x 3 steps x 131072 items x 32 bytes
-    assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 8 * 3 * 131072 * 32
-    # HIER 4 x 8 on 2 MiB: 32 ranks x 2 steps x (131072 / 8) items x 32 bytes
-    assert vrar.workspace_bytes(32, 1 << 20, torch.bfloat16, "hier") == 32 * 2 * 16384 * 32
+@pytest.mark.skipif(torch.cuda.is_available(), reason="the device-independent bound applies without a GPU")
+def test_workspace_bytes_without_a_device():
+    """Without a device the slot bytes of a shape are bounded for any grid:
+    one round over the whole message takes P x steps x items x 32 bytes, and
+    several rounds take two slot sets of fewer slots, so twice that."""
+    # RD at P=8 on 2 MiB of bf16 per rank: 8 ranks x 3 steps x 131072 items x 32 bytes, twice
+    assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "rd") == 2 * 8 * 3 * 131072 * 32
+    # HIER 4 x 8 on 2 MiB: 32 ranks x 2 steps x (131072 / 8) items x 32 bytes, twice
+    assert vrar.workspace_bytes(32, 1 << 20, torch.bfloat16, "hier") == 2 * 32 * 2 * 16384 * 32
+
+
+def test_workspace_bytes_of_algorithms_without_payloads():
     assert vrar.workspace_bytes(8, 1 << 20, torch.bfloat16, "oneshot") == 0
     assert vrar.workspace_bytes(3, 1 << 20, torch.bfloat16, "rd") == 0

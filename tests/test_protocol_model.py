@@ -1,7 +1,8 @@
 """Host-thread model of the synchronisation protocol (tests/protocol/), on the CPU.
 
 The model restates the kernels' protocol (device ticket, flag barriers,
-sequence-numbered payload words, bounded waits) with one std::thread per CTA.
+sequence-numbered payload words reused round by round in two slot sets, bounded
+waits) with one std::thread per CTA.
 These tests run it over thousands of calls of changing shape, with a missing
 rank, under ThreadSanitizer (the race check that stands in for device-side
 sanitizers, which are closed here), and with planted protocol mistakes that it
@@ -53,11 +54,14 @@ def test_protocol_has_no_data_race_under_thread_sanitizer(tmp_path):
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr[-2000:]
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5])
 def test_planted_protocol_mistakes_are_caught(tmp_path, mutant):
     """1: payload polls ignore the sequence number; 2: the ticket never returns
     its low half to 0, so calls share a flag; 3: barrier posts go to the wrong
-    words, so a barrier no longer waits for its peers."""
+    words, so a barrier no longer waits for its peers; 4: the rounds of a
+    recursive doubling share one slot set, so a writer overwrites a word its
+    reader has not read yet; 5: round tags carry no lap bit, so a reader takes
+    the word left two rounds earlier for the current one."""
     exe = _build(tmp_path, f"model_m{mutant}", "-O2", f"-DMODEL_MUTANT={mutant}")
     assert isinstance(exe, str), exe
     r = _run(exe, 300)
