@@ -21,7 +21,8 @@ import numpy as np
 
 from . import build as _build
 
-ALGOS = ("oneshot", "twostage", "twostage_write", "rd", "hier", "rd_fp32wire", "hier_fp32wire")
+ALGOS = ("oneshot", "twostage", "twostage_write", "rd", "hier", "rd_fp32wire", "hier_fp32wire",
+         "oneshot_fp8", "twostage_fp8", "twostage_write_fp8")
 _NP = {"bf16": np.uint16, "fp16": np.uint16, "fp32": np.float32}
 
 
@@ -63,6 +64,10 @@ class Oracle:
         L.oracle_all_gather.restype = ctypes.c_int
         L.oracle_fp64_reference.argtypes = [pp, ctypes.c_int, i64, cp, vp, vp]
         L.oracle_fp64_reference.restype = ctypes.c_int
+        L.oracle_e4m3_round.argtypes = [vp, vp, i64]
+        L.oracle_e4m3_round.restype = None
+        L.oracle_fp8_wire.argtypes = [vp, i64]
+        L.oracle_fp8_wire.restype = None
         self.lib = L
         self.path = path
 
@@ -92,6 +97,20 @@ class Oracle:
         h = np.ascontiguousarray(h, dtype=np.uint16)
         y = np.empty(h.shape, np.float32)
         self.lib.oracle_fp16_widen(h.ctypes.data, y.ctypes.data, h.size)
+        return y
+
+    def e4m3_round(self, x: np.ndarray) -> np.ndarray:
+        """float32 -> the nearest OCP FP8 E4M3 value (ties to even, saturating at 448), as float32."""
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        y = np.empty(x.shape, np.float32)
+        self.lib.oracle_e4m3_round(x.ctypes.data, y.ctypes.data, x.size)
+        return y
+
+    def fp8_wire(self, x: np.ndarray) -> np.ndarray:
+        """float32 values after the fp8 wire: groups of 8 from index 0, each with
+        scale amax / 448, quantised to E4M3 and dequantised."""
+        y = np.array(x, dtype=np.float32, copy=True).ravel()
+        self.lib.oracle_fp8_wire(y.ctypes.data, y.size)
         return y
 
     def allreduce(self, algo: str, xs, dtype: str = "bf16", L: int = 8, chunks: int = 4):
@@ -197,5 +216,14 @@ def to_float(x, dtype):
     return default().to_float(x, dtype)
 
 
+def e4m3_round(x):
+    return default().e4m3_round(x)
+
+
+def fp8_wire(x):
+    return default().fp8_wire(x)
+
+
 __all__ = ["ALGOS", "Oracle", "default", "allreduce", "reduce_scatter", "all_gather",
-           "fp64_reference", "bf16_round", "bf16_widen", "fp16_round", "fp16_widen", "to_float"]
+           "fp64_reference", "bf16_round", "bf16_widen", "fp16_round", "fp16_widen", "to_float", "e4m3_round",
+           "fp8_wire"]

@@ -41,11 +41,30 @@
  *    (1 sign, 5 exponent bits biased by 15, 10 fraction bits; subnormals in
  *    steps of 2^-24; values from 65520 up round to infinity); NaN -> 0x7E00.
  *
+ *  - fp8 payloads ("oneshot_fp8", "twostage_fp8", "twostage_write_fp8"; the
+ *    ca_fp8_quant flag of the custom all-reduce, whose scheme the sources do
+ *    not give - this is the reading taken): every value that passes from one
+ *    rank to another travels as OCP FP8 E4M3 (1 sign, 4 exponent bits biased
+ *    by 7, 3 fraction bits, subnormals in steps of 2^-9, no infinities,
+ *    largest finite 448) with one binary32 scale per group of 8 consecutive
+ *    elements (one 16-byte item of a 16-bit tensor; the last group holds what
+ *    is left). The scale is s = amax / 448 (amax = the largest magnitude in the
+ *    group; s = 1 if that division gives 0); an element quantises to
+ *    q = E4M3(x / s), round to nearest even, magnitudes past 448 saturating to
+ *    448, and dequantises to q * s (binary32 division and product, both round
+ *    to nearest even). One-shot quantises every input once (every rank reads
+ *    all P inputs through the fp8 wire, its own included, so that all outputs
+ *    agree); the 2-stage variants quantise the inputs for the reduce-scatter
+ *    and the reduced binary32 slice again for the all-gather, and every rank,
+ *    the owner included, stores the dequantised value rounded to the tensor
+ *    type.
+ *
  * Floating-point environment: the functions below clear the x86 flush-to-zero
  * and denormals-are-zero bits for their duration, so subnormal inputs and
  * sums are handled exactly as IEEE-754 says, whatever the caller left set.
  */
 
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <cstring>
@@ -365,6 +384,109 @@ void all_gather(const void* const* in, void* const* out, int P, int64_t n) {
             for (int64_t j = 0; j < m; ++j) out_ptr<E>(out, p)[c * m + j] = in_ptr<E>(in, c)[j];
 }
 
+
+/* ---- OCP FP8 E4M3 and the fp8 wire (readings of ca_fp8_quant) ----------------- */
+
+/* Round a binary32 to the nearest E4M3 value, ties to even, magnitudes past the
+ * largest finite value (448) saturating to it. Values are kept as binary32
+ * (every E4M3 value is exact in binary32). In the binade [2^e, 2^(e+1)) with
+ * e >= -6 the E4M3 values are spaced 2^(e-3) apart; below 2^-6 (subnormals)
+ * they are spaced 2^-9 apart. So the value is round_half_even(|v| / ulp) * ulp
+ * with that spacing; both scalings are by powers of two and exact, and the
+ * integer rounding is exact in binary32. */
+inline float e4m3_round(float v) {
+    const float a = v < 0.0f ? -v : v;
+    if (!(a == a)) return v;  /* NaN stays NaN (inputs are finite in every use) */
+    float ulp;
+    if (a < 0.015625f) {      /* below 2^-6: subnormal spacing */
+        ulp = 0.001953125f;   /* 2^-9 */
+    } else {
+        int e = 0;
+        float m = a;
+        while (m >= 2.0f) { m *= 0.5f; ++e; }
+        while (m < 1.0f) { m *= 2.0f; --e; }
+        ulp = 1.0f;
+        for (int k = 0; k < e - 3; ++k) ulp *= 2.0f;
+        for (int k = 0; k > e - 3; --k) ulp *= 0.5f;
+    }
+    const float t = a / ulp;                 /* exact: power-of-two scaling */
+    float r = static_cast<float>(static_cast<int64_t>(t));   /* floor, t >= 0 */
+    const float frac = t - r;                /* exact */
+    if (frac > 0.5f || (frac == 0.5f && std::fmod(r, 2.0f) != 0.0f)) r += 1.0f;
+    float q = r * ulp;                       /* exact */
+    if (q > 448.0f) q = 448.0f;              /* saturate (RNE may step to 480 or beyond) */
+    return v < 0.0f || (v == 0.0f && std::signbit(v)) ? -q : q;
+}
+
+/* Quantise and dequantise one group of `len` binary32 values in place. */
+inline void fp8_group_qdq(float* x, int len) {
+    float amax = 0.0f;
+    for (int i = 0; i < len; ++i) {
+        const float a = x[i] < 0.0f ? -x[i] : x[i];
+        if (a > amax) amax = a;
+    }
+    volatile float s = amax / 448.0f;
+    float sc = s;
+    if (sc == 0.0f) sc = 1.0f;
+    for (int i = 0; i < len; ++i) {
+        volatile float t = x[i] / sc;
+        volatile float d = e4m3_round(t) * sc;
+        x[i] = d;
+    }
+}
+
+/* Apply the fp8 wire to a whole vector of binary32 values: groups of 8. */
+inline void fp8_wire(std::vector<float>& v) {
+    const int64_t n = static_cast<int64_t>(v.size());
+    for (int64_t g = 0; g < n; g += 8) fp8_group_qdq(v.data() + g, static_cast<int>(n - g < 8 ? n - g : 8));
+}
+
+/* Rank p's input as binary32 after the fp8 wire. */
+template <class E>
+std::vector<float> fp8_input(const void* const* in, int p, int64_t n) {
+    std::vector<float> v(static_cast<size_t>(n));
+    for (int64_t i = 0; i < n; ++i) v[i] = E::widen(in_ptr<E>(in, p)[i]);
+    fp8_wire(v);
+    return v;
+}
+
+/* One-shot with fp8 payloads: every rank reads all P inputs through the fp8
+ * wire, adds them in ascending rank order in binary32, rounds once. */
+template <class E>
+void oneshot_fp8(const void* const* in, void* const* out, int P, int64_t n) {
+    std::vector<std::vector<float>> x(P);
+    for (int p = 0; p < P; ++p) x[p] = fp8_input<E>(in, p, n);
+    for (int r = 0; r < P; ++r)
+        for (int64_t i = 0; i < n; ++i) {
+            float acc = x[0][i];
+            for (int p = 1; p < P; ++p) acc = add32(acc, x[p][i]);
+            out_ptr<E>(out, r)[i] = E::narrow(acc);
+        }
+}
+
+/* 2-stage with fp8 payloads. Reduce-scatter: the owner of each slice adds
+ * the P inputs, each through the fp8 wire, in ascending rank order in
+ * binary32. All-gather: the reduced binary32 slice passes the fp8 wire again
+ * (groups of 8 of the vector, which never straddle two slices: slices are
+ * whole 16-byte items), and every rank stores it rounded to the tensor type.
+ * Pull and write modes store the same values. */
+template <class E>
+void twostage_fp8(const void* const* in, void* const* out, int P, int64_t n) {
+    Split sp(n, P, E::bytes);
+    std::vector<std::vector<float>> x(P);
+    for (int p = 0; p < P; ++p) x[p] = fp8_input<E>(in, p, n);
+    std::vector<float> sum(static_cast<size_t>(n));
+    for (int c = 0; c < P; ++c)
+        for (int64_t i = sp.lo(c); i < sp.hi(c); ++i) {
+            float acc = x[0][i];
+            for (int p = 1; p < P; ++p) acc = add32(acc, x[p][i]);
+            sum[i] = acc;
+        }
+    fp8_wire(sum);
+    for (int r = 0; r < P; ++r)
+        for (int64_t i = 0; i < n; ++i) out_ptr<E>(out, r)[i] = E::narrow(sum[i]);
+}
+
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 enum Dt { DT_BF16 = 0, DT_F16 = 1, DT_F32 = 2 };
@@ -409,6 +531,11 @@ int allreduce_t(const char* algo, const void* const* in, void* const* out, int P
         hier_allreduce_fp32wire<E>(in, out, P, n, L, chunks);
         return 0;
     }
+    const bool fp8 = std::strcmp(algo, "oneshot_fp8") == 0 || std::strcmp(algo, "twostage_fp8") == 0 ||
+                     std::strcmp(algo, "twostage_write_fp8") == 0;
+    if (fp8 && E::bytes != 2) return -2;  /* fp8 payloads are defined for 16-bit tensors */
+    if (std::strcmp(algo, "oneshot_fp8") == 0) { oneshot_fp8<E>(in, out, P, n); return 0; }
+    if (fp8) { twostage_fp8<E>(in, out, P, n); return 0; }
     return -1;
 }
 
@@ -439,8 +566,23 @@ void oracle_fp16_widen(const uint16_t* x, float* y, int64_t n) {
     for (int64_t i = 0; i < n; ++i) y[i] = half_widen(x[i]);
 }
 
+/* Round n binary32 values to E4M3 values (returned as binary32). */
+void oracle_e4m3_round(const float* x, float* y, int64_t n) {
+    IeeeScope env;
+    for (int64_t i = 0; i < n; ++i) y[i] = e4m3_round(x[i]);
+}
+
+/* The fp8 wire on n binary32 values (groups of 8 from index 0), in place. */
+void oracle_fp8_wire(float* x, int64_t n) {
+    IeeeScope env;
+    std::vector<float> v(x, x + n);
+    fp8_wire(v);
+    for (int64_t i = 0; i < n; ++i) x[i] = v[i];
+}
+
 /* All-reduce of P rank buffers of n elements. algo: "oneshot", "twostage",
- * "twostage_write", "rd", "hier", "rd_fp32wire", "hier_fp32wire"; dtype: "bf16" or "fp16" (uint16 bit
+ * "twostage_write", "rd", "hier", "rd_fp32wire", "hier_fp32wire", "oneshot_fp8", "twostage_fp8",
+ * "twostage_write_fp8" (the last three for bf16 / fp16 only); dtype: "bf16" or "fp16" (uint16 bit
  * patterns) or "fp32". L is the group size for "hier"; chunks is the chunk
  * count of the recursive-doubling phase. Returns 0, -1 (bad argument) or -2 (P/L shape the
  * algorithm does not define). */

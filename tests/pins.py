@@ -15,7 +15,14 @@ oracle disagrees with what the mathematics or the sources fix:
 * the error bound against math.fsum;
 * numpy's sequential float32 accumulate (a library left fold);
 * invariants the sources imply (all ranks equal; one-shot = 2-stage; chunk
-  count and special shapes reduce to the simpler algorithms).
+  count and special shapes reduce to the simpler algorithms);
+* for the fp8 payloads (the reading of the custom all-reduce's ca_fp8_quant
+  flag): E4M3 rounding against a brute-force search over every finite E4M3
+  value decoded from the format's definition (exact fractions) and against
+  torch's float8_e4m3fn cast, the group scaling and both fp8 algorithms
+  against a numpy restatement, the hand-derived case in
+  tests/golden/fp8_cases.json, exact power-of-two scale invariance and an
+  error bound.
 
 The same checks run against deliberately broken builds of the oracle, each of
 which must fail at least one of them.
@@ -24,6 +31,7 @@ which must fail at least one of them.
 from __future__ import annotations
 
 import math
+from fractions import Fraction
 
 import numpy as np
 import torch
@@ -299,6 +307,178 @@ def pin_shape_errors(o):
         raise AssertionError("hier with G=3 must be rejected")
 
 
+# ---- fp8 payloads: OCP FP8 E4M3, one binary32 scale per group of 8 -------------------------
+
+def _e4m3_values():
+    """Every finite non-negative E4M3 value with its code, decoded from the
+    format: 1 sign bit, 4 exponent bits biased by 7, 3 fraction bits; exponent
+    field 0 holds the subnormals frac/8 * 2^-6; code 0x7F (all ones) is NaN and
+    there are no infinities."""
+    out = []
+    for code in range(0x7F):
+        e, f = code >> 3, code & 7
+        v = Fraction(f, 8) * Fraction(1, 64) if e == 0 else (1 + Fraction(f, 8)) * Fraction(2) ** (e - 7)
+        out.append((v, code))
+    return out
+
+
+_E4M3 = _e4m3_values()
+
+
+def e4m3_brute(x: float) -> float:
+    """Nearest E4M3 value to x by exhaustive search over the finite values
+    (saturating past the largest, 448); ties go to the even code."""
+    a = Fraction(abs(float(x)))
+    best = min(_E4M3, key=lambda vc: (abs(vc[0] - a), vc[1] & 1))
+    v = float(best[0])
+    return -v if math.copysign(1.0, float(x)) < 0 else v
+
+
+def _e4m3_torch(t32: np.ndarray) -> np.ndarray:
+    """torch's float32 -> float8_e4m3fn cast (round to nearest even) and back."""
+    return torch.from_numpy(t32).to(torch.float8_e4m3fn).to(torch.float32).numpy()
+
+
+def fp8_wire_numpy(x32: np.ndarray) -> np.ndarray:
+    """The fp8 wire restated in numpy: groups of 8 from index 0; s = amax / 448
+    in binary32 (1 if that is 0); q = E4M3(x / s) with torch's cast; q * s in
+    binary32. A binary32 quotient or product formed in float64 and then
+    rounded to binary32 is the correctly rounded binary32 result (53 >= 2*24+2
+    bits), so these match IEEE binary32 division and multiplication."""
+    x = np.asarray(x32, np.float32)
+    out = np.empty_like(x)
+    for g in range(0, x.size, 8):
+        grp = x[g:g + 8]
+        amax = np.float32(np.max(np.abs(grp))) if grp.size else np.float32(0)
+        s = np.float32(np.float64(amax) / 448.0)
+        if s == 0:
+            s = np.float32(1.0)
+        t = (grp.astype(np.float64) / np.float64(s)).astype(np.float32)
+        q = _e4m3_torch(t)
+        out[g:g + 8] = (q.astype(np.float64) * np.float64(s)).astype(np.float32)
+    return out
+
+
+def _to32(x, dtype):
+    if dtype == "bf16":
+        return (x.astype(np.uint32) << 16).view(np.float32)
+    return x.view(np.float16).astype(np.float32)
+
+
+def _round_to(y32, dtype):
+    if dtype == "bf16":
+        return to_np(torch.from_numpy(np.ascontiguousarray(y32)).to(torch.bfloat16))
+    return np.ascontiguousarray(y32).astype(np.float16).view(np.uint16)
+
+
+def pin_e4m3_round_brute(o):
+    pts = []
+    vals = sorted(v for v, _ in _E4M3)
+    for a, b in zip(vals, vals[1:]):
+        mid = (a + b) / 2
+        m = np.float32(float(mid))
+        assert Fraction(float(m)) == mid, "E4M3 midpoints are exact in binary32"
+        pts += [m, np.nextafter(m, np.float32(0)), np.nextafter(m, np.float32(1e9)), np.float32(float(a))]
+    pts += [np.float32(v) for v in (448.0, 450.0, 463.99, 464.0, 470.0, 480.0, 1e4, 3e38, 0.0, 2.0**-10,
+                                     2.0**-11, 3 * 2.0**-10, 2.0**-9, 2.0**-20, 1e-40)]
+    rng = np.random.default_rng(8)
+    pts += list((2.0 ** rng.uniform(-14, 9.2, 1500)).astype(np.float32))
+    x = np.array(pts, np.float32)
+    x = np.concatenate([x, -x])
+    got = o.e4m3_round(x)
+    want = np.array([e4m3_brute(v) for v in x], np.float32)
+    bad = np.nonzero(got.view(np.uint32) != want.view(np.uint32))[0]
+    assert bad.size == 0, f"E4M3 rounding differs at {x[bad[:5]]}: {got[bad[:5]]} vs {want[bad[:5]]}"
+
+
+def pin_e4m3_round_vs_torch(o):
+    rng = np.random.default_rng(9)
+    x = (rng.uniform(-1, 1, 200_000) * 2.0 ** rng.uniform(-16, 8.85, 200_000)).astype(np.float32)
+    x = x[np.abs(x) < 464]  # torch's cast gives NaN from the rounding boundary past 448 on; ours saturates
+    got, want = o.e4m3_round(x), _e4m3_torch(x)
+    assert (got.view(np.uint32) == want.view(np.uint32)).all(), "E4M3 rounding differs from torch's cast"
+
+
+def pin_fp8_wire_numpy(o):
+    rng = np.random.default_rng(10)
+    cases = [rng.normal(0, 1, 531).astype(np.float32),
+             (rng.normal(0, 1, 64) * 2.0 ** rng.integers(-30, 30, 64)).astype(np.float32),
+             np.zeros(16, np.float32), np.array([-0.0] * 5 + [1e-3] * 3, np.float32),
+             np.array([448.0, 1e-6, -2e-5, 3e-4, 0, 5, 6, 7, 1e-30, 2e-30, -3e-30], np.float32)]
+    bits = rng.integers(0, 1 << 16, 200, dtype=np.uint32)          # raw bf16 patterns, incl. subnormals
+    bits = bits[(bits & 0x7F80) != 0x7F80]                          # finite ones
+    cases.append((bits << 16).view(np.float32))
+    for x in cases:
+        got, want = o.fp8_wire(x), fp8_wire_numpy(x)
+        assert (got.view(np.uint32) == want.view(np.uint32)).all(), "fp8 wire differs from the numpy restatement"
+
+
+def pin_fp8_allreduce_numpy(o):
+    for dtype in ("bf16", "fp16"):
+        for P in (1, 2, 3, 8):
+            n = 531
+            xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=800 + P)
+            wired = [fp8_wire_numpy(_to32(x, dtype)) for x in xs]
+            acc = wired[0].copy()
+            for w in wired[1:]:
+                acc = (acc + w).astype(np.float32)  # one binary32 add per element, ascending rank order
+            one = _round_to(acc, dtype)
+            two = _round_to(fp8_wire_numpy(acc), dtype)
+            for algo, want in (("oneshot_fp8", one), ("twostage_fp8", two), ("twostage_write_fp8", two)):
+                outs = o.allreduce(algo, xs, dtype)
+                assert _all_equal(outs), f"{algo}: ranks differ"
+                assert (bits_of(outs[0]) == bits_of(want)).all(), f"{algo} {dtype} P={P}: differs from numpy"
+
+
+def pin_fp8_golden(o):
+    for c in load_golden("fp8_cases.json")["cases"]:
+        xs = [hexvals(r, c["dtype"]) for r in c["inputs"]]
+        for algo, key in (("oneshot_fp8", "oneshot_fp8"), ("twostage_fp8", "twostage_fp8"),
+                          ("twostage_write_fp8", "twostage_fp8")):
+            want = hexvals(c[key], c["dtype"])
+            for p, out in enumerate(o.allreduce(algo, xs, c["dtype"])):
+                assert (bits_of(out) == bits_of(want)).all(), f"{c['name']} {algo} rank {p}"
+
+
+def pin_fp8_invariants(o):
+    rng = np.random.default_rng(11)
+    x = rng.normal(0, 1, 1000).astype(np.float32)
+    base = o.fp8_wire(x)
+    for k in (-20, -7, -1, 1, 5, 20):  # power-of-two scaling is exact at every step
+        scaled = o.fp8_wire((x * np.float32(2.0 ** k)).astype(np.float32))
+        assert (scaled == (base * np.float32(2.0 ** k)).astype(np.float32)).all(), f"not scale invariant (2^{k})"
+    # Groups whose largest magnitude is 448 and whose values are E4M3 values
+    # have scale 1 and pass unchanged, so one-shot over them is the plain one-shot.
+    vals = np.array(sorted({float(v) for v, _ in _E4M3}), np.float32)
+    for dtype in ("bf16", "fp16"):
+        xs = []
+        for p in range(4):
+            g = rng.choice(np.concatenate([vals, -vals]), size=(40, 8)).astype(np.float32)
+            g[:, rng.integers(0, 8)] = 448.0 * (1 if p % 2 else -1)
+            xs.append(_round_to(g.ravel(), dtype))
+        assert (bits_of(o.allreduce("oneshot_fp8", xs, dtype)[0]) == bits_of(o.allreduce("oneshot", xs, dtype)[0])).all()
+    # Error bound: each dequantised value is within 2^-4 of its input relative
+    # (E4M3 keeps 4 significant bits) plus 2^-10 of the group scale (the
+    # subnormal spacing), and the fp32 adds and the final rounding add less
+    # than 2^-8 of the magnitudes; the 2-stage wire adds the same again on the sum.
+    xs = gen(8, 4099, "bf16", synth.normal(0.0, 1.0), seed=12)
+    S, A = o.fp64_reference(xs, "bf16")
+    amax_sum = sum(np.repeat(np.abs(_to32(x, "bf16")).reshape(-1, 1)[:4096].reshape(-1, 8).max(axis=1), 8)[:4096]
+                   for x in xs)
+    y1 = o.to_float(o.allreduce("oneshot_fp8", xs, "bf16")[0], "bf16")[:4096]
+    y2 = o.to_float(o.allreduce("twostage_fp8", xs, "bf16")[0], "bf16")[:4096]
+    bound1 = (2.0**-4 + 2.0**-8) * A[:4096] + 2.0**-10 / 448 * 1.01 * amax_sum
+    assert (np.abs(y1 - S[:4096]) <= bound1).all(), "oneshot_fp8 outside its error bound"
+    assert (np.abs(y2 - S[:4096]) <= 2 * bound1 + 2.0**-4 * np.abs(S[:4096])).all(), "twostage_fp8 outside its bound"
+    for algo in ("oneshot_fp8", "twostage_fp8"):
+        try:
+            o.allreduce(algo, gen(2, 8, "fp32", synth.INT8), "fp32")
+        except ValueError:
+            pass
+        else:
+            raise AssertionError(f"{algo} must reject fp32 elements")
+
+
 ALL_PINS = [
     pin_bf16_round_vs_torch,
     pin_bf16_round_hand,
@@ -314,4 +494,10 @@ ALL_PINS = [
     pin_invariants,
     pin_rs_ag,
     pin_shape_errors,
+    pin_e4m3_round_brute,
+    pin_e4m3_round_vs_torch,
+    pin_fp8_wire_numpy,
+    pin_fp8_allreduce_numpy,
+    pin_fp8_golden,
+    pin_fp8_invariants,
 ]

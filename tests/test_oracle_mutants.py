@@ -50,6 +50,18 @@ MUTANTS = {
         "part[g * L + l][i] = E::widen(reduce_ranks<E>(in, g * L, L, i));"),
     "half_widen_bias": ("return bits_to_f32(sign | ((exp + 112u) << 23) | (frac << 13));",
                         "return bits_to_f32(sign | ((exp + 111u) << 23) | (frac << 13));"),
+    "e4m3_round_half_away": ("if (frac > 0.5f || (frac == 0.5f && std::fmod(r, 2.0f) != 0.0f)) r += 1.0f;",
+                             "if (frac >= 0.5f) r += 1.0f;"),
+    "e4m3_truncate": ("if (frac > 0.5f || (frac == 0.5f && std::fmod(r, 2.0f) != 0.0f)) r += 1.0f;",
+                      "if (frac > 2.0f) r += 1.0f;"),
+    "e4m3_flush_subnormals": ("ulp = 0.001953125f;   /* 2^-9 */", "ulp = 0.015625f;"),
+    "e4m3_no_saturation": ("if (q > 448.0f) q = 448.0f;", ""),
+    "fp8_scale_fnuz_max": ("volatile float s = amax / 448.0f;", "volatile float s = amax / 240.0f;"),
+    "fp8_amax_signed": ("const float a = x[i] < 0.0f ? -x[i] : x[i];\n        if (a > amax) amax = a;",
+                        "const float a = x[i];\n        if (a > amax) amax = a;"),
+    "fp8_groups_of_4": ("for (int64_t g = 0; g < n; g += 8) fp8_group_qdq(v.data() + g, static_cast<int>(n - g < 8 ? n - g : 8));",
+                        "for (int64_t g = 0; g < n; g += 4) fp8_group_qdq(v.data() + g, static_cast<int>(n - g < 4 ? n - g : 4));"),
+    "twostage_fp8_single_wire": ("    fp8_wire(sum);\n", ""),
 }
 
 
