@@ -75,10 +75,11 @@ PER_ALGO_STEPS = 10     # graph length of the per-algorithm rows on the headline
 SWEEP = (
     [dict(DECODE, algos=("oneshot", "twostage", "twostage_write", "rd", "auto"), collectives=("rs", "ag"),
           warm=("auto", "oneshot", "twostage", "twostage_write", "rd"),
-          edge=("oneshot", "twostage_write"))]
+          edge=("oneshot", "twostage_write"), fp8=("oneshot", "twostage", "twostage_write"))]
     + [dict(name=f"P=8 sweep {b >> 10} KiB per rank, N(0,1)", P=8, n=b // 2, dtype="bf16", dist="normal:0,1",
             algos=("oneshot", "twostage", "twostage_write", "rd", "auto"), collectives=("rs", "ag"),
-            edge=("oneshot", "twostage_write") if b == 2 << 20 else ())
+            edge=("oneshot", "twostage_write") if b == 2 << 20 else (),
+            fp8=("oneshot", "twostage_write") if b == 2 << 20 else ())
        for b in (128 << 10, 256 << 10, 512 << 10, 2 << 20)]
     + [dict(name="P=2 ints 128 KiB per rank", P=2, n=65536, dtype="bf16", dist="int8",
             algos=("oneshot", "rd", "auto"))]
@@ -583,38 +584,50 @@ def oracle_samples(spec, algo: str, min_seconds: float, n_sample: int, device=No
 
 # ---- arms -------------------------------------------------------------------------------------------
 
-def with_edge(algo: str):
-    """'twostage_write+edge' -> ('twostage_write', True): the algorithm with the
-    start/end barriers on."""
-    return (algo[:-5], True) if algo.endswith("+edge") else (algo, False)
+def with_flags(algo: str):
+    """'twostage_write+edge+fp8' -> ('twostage_write', edge=True, fp8=True): the
+    algorithm with the start/end barriers and / or the fp8 payloads on."""
+    parts = algo.split("+")
+    return parts[0], "edge" in parts[1:], "fp8" in parts[1:]
+
+
+class flags_set:
+    """Turn the settings a row's suffixes name on for its capture (a graph keeps
+    the settings its calls were queued with), and back off after."""
+
+    def __init__(self, vrar, algo):
+        self.vrar, (self.base, self.edge, self.fp8) = vrar, with_flags(algo)
+
+    def __enter__(self):
+        self.vrar.set_edge_sync(self.edge)
+        self.vrar.set_fp8_quant(self.fp8)
+        return self.base
+
+    def __exit__(self, *exc):
+        self.vrar.set_edge_sync(False)
+        self.vrar.set_fp8_quant(False)
 
 
 def measure_row(vrar, w: Workload, algo: str, steps: int, warmup: int, world, device, replays: int):
-    base, edge = with_edge(algo)
-    vrar.set_edge_sync(edge)  # read when a call is queued: the graph keeps it
-    try:
+    with flags_set(vrar, algo) as base:
         return measure_algo(w, base, steps, warmup, world, device, replays)
-    finally:
-        vrar.set_edge_sync(False)
 
 
 def spin_row(vrar, w: Workload, algo: str, calls: int) -> dict:
     """Spin statistics of the waits of `calls` calls (a separate, instrumented
     graph: the counters cost a few atomics per warp and wait, so the timed rows
     run without them)."""
-    base, edge = with_edge(algo)
-    vrar.set_edge_sync(edge)
-    vrar.set_spin_stats(True)
-    try:
-        w.call(0, base, torch.cuda.current_stream().cuda_stream)
-        torch.cuda.synchronize()
-        g = w.graph(base, calls)
-        vrar.get_spin_stats(reset=True)
-        g.replay()
-        torch.cuda.synchronize()
-    finally:
-        vrar.set_spin_stats(False)
-        vrar.set_edge_sync(False)
+    with flags_set(vrar, algo) as base:
+        vrar.set_spin_stats(True)
+        try:
+            w.call(0, base, torch.cuda.current_stream().cuda_stream)
+            torch.cuda.synchronize()
+            g = w.graph(base, calls)
+            vrar.get_spin_stats(reset=True)
+            g.replay()
+            torch.cuda.synchronize()
+        finally:
+            vrar.set_spin_stats(False)
     st = vrar.get_spin_stats(reset=True)
     rc, _ = vrar.query_status()
     del g
@@ -649,9 +662,9 @@ def run_vrar(args):
 
     per_algo = {}
     if not args.quick:
-        for algo in ("oneshot", "twostage", "twostage_write", "rd"):
-            per_algo[algo] = entry(wl, measure_algo(wl, algo, PER_ALGO_STEPS, 3, world, device, 3) / 1e3, peak,
-                                   algo)
+        for algo in ("oneshot", "twostage", "twostage_write", "rd", "twostage_write+fp8", "oneshot+fp8"):
+            per_algo[algo] = entry(wl, measure_row(vrar, wl, algo, PER_ALGO_STEPS, 3, world, device, 3) / 1e3,
+                                   peak, with_flags(algo)[0])
         for kind in ("rs", "ag"):
             t = measure_collective(wl, kind, PER_ALGO_STEPS, 3, world, device, 3) / 1e3
             ach = (wl.P + 1) * wl.n * wl.esz / t / 1e9  # (P + 1) n s either way
@@ -681,6 +694,10 @@ def run_vrar(args):
                 row[key] = entry(w, measure_row(vrar, w, key, 200, 3, world, device, SWEEP_REPLAYS) / 1e3, peak,
                                  algo)
                 row[key]["spin"] = spin_row(vrar, w, key, 1000)
+            for algo in spec.get("fp8", ()):
+                key = f"{algo}+fp8"
+                row[key] = entry(w, measure_row(vrar, w, key, 200, 3, world, device, SWEEP_REPLAYS) / 1e3, peak,
+                                 algo)
             for kind in spec.get("collectives", ()):
                 # RS moves P*n*s in and n*s out; AG n*s in and P*n*s out: (P+1)*n*s either way.
                 t = measure_collective(w, kind, spec.get("steps", 200), 3, world, device, SWEEP_REPLAYS) / 1e3
@@ -861,6 +878,52 @@ def run_spin_stats(args):
     vrar.set_edge_sync(False)
 
 
+def run_floor(args):
+    """Where the time of a small call goes (JSON lines). For P = 2 and 8 ranks:
+    the per-call cost of a call on one 16-byte item per rank (launch, one
+    DRAM round trip, the tail), and calls from 8 KiB to 8 MiB per rank, cold
+    (inputs rotated through more than 3x L2) and warm (one buffer set, so the
+    working set stays in L2), each the median of graph replays of 1000 (small)
+    or 200 back-to-back calls. The write-mode kernel is whichever this process
+    runs (VRAR_WRITE_KERNEL forces one). A straight-line fit of the cold times
+    from 512 KiB per rank up, t = t0 + B_min / BW, splits each call into a
+    fixed part t0 and a streaming part."""
+    import collective_all_reduce_virtual_b200 as vrar
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    kernel = os.environ.get("VRAR_WRITE_KERNEL", "auto")
+    for P in (2, 8):
+        tiny = Workload(dict(DECODE, P=P, n=8, name="one item"), device)
+        row = {"P": P, "write_kernel": kernel, "one_item_us": {}}
+        for algo in ("oneshot", "twostage_write", "twostage", "rd"):
+            row["one_item_us"][algo] = round(measure_algo(tiny, algo, 1000, 3, replays=5) * 1e3, 3)
+        tiny.free()
+        pts = []
+        for kib in (8, 32, 128, 512, 1024, 2048, 4096, 8192):
+            n = kib * 512
+            spec = dict(DECODE, P=P, n=n, name=f"P={P} {kib} KiB")
+            steps = 1000 if kib <= 512 else 200
+            cold, warm = Workload(spec, device), Workload(spec, device, rotate=False)
+            e = {"kib": kib, "bmin_bytes": b_min_bytes(P, n, 2),
+                 "kernel": vrar.kernel_name(P, n, TDT["bf16"], "auto")}
+            for algo in ("oneshot", "twostage_write"):
+                e[algo] = {"cold_us": round(measure_algo(cold, algo, steps, 3, replays=5) * 1e3, 3),
+                           "warm_us": round(measure_algo(warm, algo, steps, 3, replays=5) * 1e3, 3)}
+            cold.free()
+            warm.free()
+            torch.cuda.empty_cache()
+            pts.append(e)
+        row["sizes"] = pts
+        for algo in ("oneshot", "twostage_write"):
+            xs = [p["bmin_bytes"] for p in pts if p["kib"] >= 512]
+            ys = [p[algo]["cold_us"] * 1e-6 for p in pts if p["kib"] >= 512]
+            mx, my = sum(xs) / len(xs), sum(ys) / len(ys)
+            slope = sum((x - mx) * (y - my) for x, y in zip(xs, ys)) / sum((x - mx) ** 2 for x in xs)
+            row[f"fit_{algo}"] = {"t0_us": round((my - slope * mx) * 1e6, 3),
+                                  "stream_gbs": round(1 / slope / 1e9, 1) if slope > 0 else None}
+        print(json.dumps(row), flush=True)
+
+
 class TboPrefill:
     """Two micro-batches of a 16k-token prefill through L row-parallel linear
     layers with P virtual ranks. In each layer rank p multiplies its K/P slice
@@ -986,11 +1049,16 @@ def main(argv=None):
                     help="spin statistics of the waits over CALLS calls per algorithm (JSON lines) and exit")
     ap.add_argument("--overlap", action="store_true",
                     help="sequential vs overlapped two-micro-batch prefill step (JSON line) and exit")
+    ap.add_argument("--floor", action="store_true",
+                    help="per-call fixed cost and size ladder at 2 and 8 ranks (JSON lines) and exit")
     ap.add_argument("--selector-sweep", action="store_true",
                     help="print per-shape timings of every algorithm (JSON lines) and exit")
     args = ap.parse_args(argv)
     if args.selector_sweep:
         run_selector_sweep(args)
+        return
+    if args.floor:
+        run_floor(args)
         return
     if args.case:
         sys.exit(1 if run_case(args.case) else 0)

@@ -48,6 +48,8 @@ SIGNATURES = {
     "vrar_get_rd_chunks": ([], _i),
     "vrar_set_payload_wire": ([_i], _i),
     "vrar_get_payload_wire": ([], _i),
+    "vrar_set_fp8_quant": ([_i], _i),
+    "vrar_get_fp8_quant": ([], _i),
     "vrar_set_edge_sync": ([_i], _i),
     "vrar_get_edge_sync": ([], _i),
     "vrar_set_max_ctas": ([_i], _i),
@@ -213,6 +215,15 @@ def get_payload_wire() -> str:
     return "fp32" if _lib.vrar_get_payload_wire() == WIRE_FP32 else "element"
 
 
+def set_fp8_quant(on: bool) -> None:
+    """fp8 payloads of the custom all-reduce algorithms (see vrar_set_fp8_quant)."""
+    _check(_lib.vrar_set_fp8_quant(1 if on else 0), "vrar_set_fp8_quant")
+
+
+def get_fp8_quant() -> bool:
+    return bool(_lib.vrar_get_fp8_quant())
+
+
 def set_edge_sync(on: bool) -> None:
     _check(_lib.vrar_set_edge_sync(1 if on else 0), "vrar_set_edge_sync")
 
@@ -284,7 +295,8 @@ def version() -> int:
 
 
 __all__ = ["all_reduce", "reduce_scatter", "all_gather", "select_algo", "kernel_name", "set_group_size",
-           "get_group_size", "set_rd_chunks", "get_rd_chunks", "set_payload_wire", "get_payload_wire", "set_edge_sync", "get_edge_sync",
+           "get_group_size", "set_rd_chunks", "get_rd_chunks", "set_payload_wire", "get_payload_wire", "set_fp8_quant",
+           "get_fp8_quant", "set_edge_sync", "get_edge_sync",
            "set_max_ctas", "get_max_ctas", "set_spin_timeout_ns", "get_spin_timeout_ns", "query_status", "reserve",
            "workspace_bytes", "reset", "set_spin_stats", "get_spin_stats", "debug_set_fault_mask", "strerror", "version", "VrarError",
            "ALGOS", "DTYPES", "SIGNATURES", "LIB_PATH", "lib", "ptr_array"]

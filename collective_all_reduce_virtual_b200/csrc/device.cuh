@@ -282,8 +282,76 @@ struct F32T {
   __device__ __forceinline__ static E f_to_elem(float f) { return f; }
 };
 
+// ---- fp8 payloads (a reading of the custom all-reduce's ca_fp8_quant flag) ----------------
+// Every value that passes from one rank to another travels as OCP FP8 E4M3
+// with one binary32 scale per group of 8 elements, which is one 16-byte item
+// of a 16-bit tensor: s = amax / 448 (amax the group's largest magnitude; 1 if
+// the division gives 0), q = E4M3(x / s) rounded to nearest even and saturated
+// at 448, and the receiver's value is q * s. On one device the values never
+// need to be stored in fp8: each kernel quantises and dequantises in
+// registers where the value would cross between ranks, and moves the same
+// bytes as without fp8.
+
+// E4M3 rounding of two binary32 values and back: cvt.rn.satfinite.e4m3x2.f32
+// packs (hi, lo) into two bytes; cvt.rn.f16x2.e4m3x2 widens them exactly to
+// two halves (every E4M3 value is a binary16 value), which widen exactly to
+// binary32.
+__device__ __forceinline__ void e4m3_round2(float& lo, float& hi) {
+  uint16_t q;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(q) : "f"(hi), "f"(lo));
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(q));
+  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+// E4M3(x / s) needs the binary32 quotient x / s only up to which side of an
+// E4M3 rounding midpoint it falls. The product t = x * r with r = 1/s (both
+// rounded to nearest) is within 3 units in the last place of the quotient
+// (two roundings of 2^-24 relative each, for r a normal number), so it rounds
+// to the same E4M3 value unless a midpoint lies within 3 units of it. Where t
+// is within 8 units of a midpoint of a normal E4M3 binade (its 20 fraction bits
+// below the 3 that E4M3 keeps are within 8 of 1000...0), or in E4M3's
+// subnormal range (below 2^-6, where the midpoints sit elsewhere), the exact
+// quotient is taken instead. Binade edges are E4M3 values, not midpoints, so
+// a t on the other side of one from the quotient still rounds the same way.
+__device__ __forceinline__ float fp8_quotient(float x, float s, float r) {
+  const float t = __fmul_rn(x, r);
+  const uint32_t u = __float_as_uint(t) & 0x7FFFFFFFu;
+  const int32_t below = static_cast<int32_t>(u & 0xFFFFFu) - 0x80000;
+  if ((u != 0u && u < 0x3C800000u) || (below >= -8 && below <= 8)) return __fdiv_rn(x, s);
+  return t;
+}
+
+// The fp8 wire on one group of 8 binary32 values, in place: s = amax / 448
+// (1 when that is 0), each value quantised to E4M3(x / s) and received as
+// E4M3 * s, with binary32 division and product rounded to nearest even
+// (__fdiv_rn, __fmul_rn; the quotient as fp8_quotient gives it). Scales
+// outside [2^-125, 2^125] (whose reciprocal is not a normal number) divide
+// every value exactly.
+__device__ __forceinline__ void fp8_qdq8(float (&f)[8]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  float s = __fdiv_rn(amax, 448.0f);
+  if (s == 0.0f) s = 1.0f;
+  const bool fast = s >= 0x1p-125f && s <= 0x1p125f;
+  const float r = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    float lo = fast ? fp8_quotient(f[i], s, r) : __fdiv_rn(f[i], s);
+    float hi = fast ? fp8_quotient(f[i + 1], s, r) : __fdiv_rn(f[i + 1], s);
+    e4m3_round2(lo, hi);
+    f[i] = __fmul_rn(lo, s);
+    f[i + 1] = __fmul_rn(hi, s);
+  }
+}
+
 // fp32 accumulator of one item. Every add is add.rn.f32: round to nearest
 // even, never contracted into an FMA, subnormals kept (no .ftz).
+// init_in / add_in take an input item as it arrives from a rank (through the
+// fp8 wire when kQ8); round_out rounds the sum for an all-gather that crosses
+// ranks (through the fp8 wire again when kQ8).
 template <class D>
 struct Acc {
   float v[D::VE];
@@ -295,6 +363,32 @@ struct Acc {
     for (int i = 0; i < D::VE; ++i) v[i] = __fadd_rn(v[i], f[i]);
   }
   __device__ __forceinline__ uint4 round() const { return D::narrow(v); }
+
+  template <bool kQ8>
+  __device__ __forceinline__ void init_in(const uint4& x) {
+    D::widen(x, v);
+    if constexpr (kQ8) fp8_qdq8(v);
+  }
+  template <bool kQ8>
+  __device__ __forceinline__ void add_in(const uint4& x) {
+    float f[D::VE];
+    D::widen(x, f);
+    if constexpr (kQ8) fp8_qdq8(f);
+#pragma unroll
+    for (int i = 0; i < D::VE; ++i) v[i] = __fadd_rn(v[i], f[i]);
+  }
+  template <bool kQ8>
+  __device__ __forceinline__ uint4 round_out() const {
+    if constexpr (kQ8) {
+      float t[D::VE];
+#pragma unroll
+      for (int i = 0; i < D::VE; ++i) t[i] = v[i];
+      fp8_qdq8(t);
+      return D::narrow(t);
+    } else {
+      return D::narrow(v);
+    }
+  }
 };
 
 // rnd(f(a) + f(b)) element-wise: one recursive-doubling combine.
@@ -348,13 +442,15 @@ __device__ __forceinline__ void store_item(void* base, int64_t it, int64_t n, co
   }
   union { uint4 u; typename D::E e[D::VE]; } t;
   t.u = v;
-  for (int i = 0; i < nv; ++i) p[i] = t.e[i];
+#pragma unroll
+  for (int i = 0; i < D::VE; ++i)
+    if (i < nv) p[i] = t.e[i];
 }
 
 // Ascending-rank fp32 sum of item `it` over ranks first .. first+count-1 (not
-// rounded). Loads are issued eight at a time so that they overlap; the adds
-// stay in rank order.
-template <class D>
+// rounded), each input through the fp8 wire when kQ8. Loads are issued eight
+// at a time so that they overlap; the adds stay in rank order.
+template <class D, bool kQ8 = false>
 __device__ __forceinline__ Acc<D> reduce_item_acc(const RankPtrs& rp, int first, int count, int64_t it, int64_t n) {
   Acc<D> acc;
   for (int q0 = 0; q0 < count; q0 += 8) {
@@ -365,7 +461,7 @@ __device__ __forceinline__ Acc<D> reduce_item_acc(const RankPtrs& rp, int first,
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (q0 + j < count) {
-        if (q0 + j == 0) acc.init(x[j]); else acc.add(x[j]);
+        if (q0 + j == 0) acc.template init_in<kQ8>(x[j]); else acc.template add_in<kQ8>(x[j]);
       }
     }
   }
@@ -373,9 +469,16 @@ __device__ __forceinline__ Acc<D> reduce_item_acc(const RankPtrs& rp, int first,
 }
 
 // The same sum rounded once to the element type.
-template <class D>
+template <class D, bool kQ8 = false>
 __device__ __forceinline__ uint4 reduce_item(const RankPtrs& rp, int first, int count, int64_t it, int64_t n) {
-  return reduce_item_acc<D>(rp, first, count, it, n).round();
+  return reduce_item_acc<D, kQ8>(rp, first, count, it, n).round();
+}
+
+// The sum as the 2-stage kernels hand it to the other ranks: through the fp8
+// wire a second time when kQ8, then rounded to the element type.
+template <class D, bool kQ8>
+__device__ __forceinline__ uint4 reduce_item_out(const RankPtrs& rp, int first, int count, int64_t it, int64_t n) {
+  return reduce_item_acc<D, kQ8>(rp, first, count, it, n).template round_out<kQ8>();
 }
 
 // A 16-byte item of a 16-bit type as fp32 partials: two quads of 4 floats.
@@ -494,7 +597,7 @@ __device__ __forceinline__ void record_spins(const KArgs& a, uint32_t spins, boo
   }
 }
 
-__device__ __noinline__ void report_timeout(const KArgs& a, const Cta& c, uint32_t phase) {
+__device__ __forceinline__ void report_timeout(const KArgs& a, const Cta& c, uint32_t phase) {
   if (atomicCAS(a.ctrl + kStatus, 0u, kErrTimeout) == 0u) {
     a.ctrl[kInfo + 0] = c.flag;
     a.ctrl[kInfo + 1] = phase;

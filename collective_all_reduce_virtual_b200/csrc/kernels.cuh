@@ -27,8 +27,9 @@ __device__ __forceinline__ int64_t lo_of(int64_t part, int64_t piece, int64_t to
 // reduces the whole vector into its own output, between start and end
 // barriers. The P CTAs with the same b read the same items at about the same
 // time, so all but the first read of each line hit L2. T threads per CTA:
-// small messages run faster as more, smaller CTAs.
-template <class D, int T = kThreads>
+// small messages run faster as more, smaller CTAs. kQ8: every input passes
+// the fp8 wire once (every rank reads all P inputs through it).
+template <class D, int T = kThreads, bool kQ8 = false>
 __global__ void __launch_bounds__(T, 2) k_oneshot(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
@@ -43,7 +44,7 @@ __global__ void __launch_bounds__(T, 2) k_oneshot(const KArgs a) {
   const int64_t stride = static_cast<int64_t>(a.B) * T;
   void* out = a.ptr.out[c.r];
   for (int64_t it = static_cast<int64_t>(c.b) * T + threadIdx.x; it < a.items; it += stride)
-    store_item<D, true>(out, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
+    store_item<D, true>(out, it, a.n, reduce_item<D, kQ8>(a.ptr, 0, a.P, it, a.n));
   if (a.edge_sync) block_barrier(a, c, kPhEnd);
 }
 
@@ -51,7 +52,9 @@ __global__ void __launch_bounds__(T, 2) k_oneshot(const KArgs a) {
 // reduces slice r (ceil(items / P) items) over all P inputs into out[r]. Mid
 // barrier. Stage 2: rank r copies every other slice s out of out[s]. T threads
 // per CTA (the library launches 256: more, smaller CTAs per column barrier).
-template <class D, int T = kThreads>
+// kQ8: the inputs pass the fp8 wire for stage 1 and the reduced slice passes
+// it again for stage 2; the owner stores that value too.
+template <class D, int T = kThreads, bool kQ8 = false>
 __global__ void __launch_bounds__(T) k_twostage(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(T) k_twostage(const KArgs a) {
   {
     const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
     for (int64_t it = lo + t0; it < hi; it += stride)
-      store_item<D, false>(own, it, a.n, reduce_item<D>(a.ptr, 0, a.P, it, a.n));
+      store_item<D, false>(own, it, a.n, reduce_item_out<D, kQ8>(a.ptr, 0, a.P, it, a.n));
   }
   if (!a.edge_sync) cta_publish_flag(c, ticket);
   if (!block_barrier(a, c, kPhMid)) return;
@@ -102,8 +105,8 @@ __global__ void __launch_bounds__(T) k_twostage(const KArgs a) {
 // 2-stage write mode [CAR "cross_device_reduce_2stage_write_mode", Root cause
 // and change 3]: rank r reduces slice r and streams the result straight into
 // all P outputs; a device-scope fence then makes those stores visible before
-// the end barrier's flags.
-template <class D>
+// the end barrier's flags. kQ8: inputs and reduced slice pass the fp8 wire.
+template <class D, bool kQ8 = false>
 __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
   const int64_t piece = (a.items + a.P - 1) / a.P;
   const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
   for (int64_t it = lo + static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < hi; it += stride) {
-    const uint4 v = reduce_item<D>(a.ptr, 0, a.P, it, a.n);
+    const uint4 v = reduce_item_out<D, kQ8>(a.ptr, 0, a.P, it, a.n);
     for (int j = 0; j < a.P; ++j) {
       const int p = (c.r + j) % a.P;
       store_item<D, true>(a.ptr.out[p], it, a.n, v);
@@ -169,7 +172,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
-template <class D, int kStageItems>
+template <class D, int kStageItems, bool kQ8 = false>
 __global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(const KArgs a) {
   constexpr uint32_t kStageTileBytes = kStageItems * 16;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -249,9 +252,9 @@ __global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(cons
       if (base + ci < hi_full) {
         const unsigned char* src = stage0 + st * stage_bytes + ci * 16;
         Acc<D> acc;
-        acc.init(ld_shared_v4(src));
-        for (int p = 1; p < a.P; ++p) acc.add(ld_shared_v4(src + p * kStageTileBytes));
-        const uint4 v = acc.round();
+        acc.template init_in<kQ8>(ld_shared_v4(src));
+        for (int p = 1; p < a.P; ++p) acc.template add_in<kQ8>(ld_shared_v4(src + p * kStageTileBytes));
+        const uint4 v = acc.template round_out<kQ8>();
         for (int j = 0; j < a.P; ++j) {
           const int q = (c.r + j) % a.P;
           st_stream(static_cast<typename D::E*>(a.ptr.out[q]) + (base + ci) * D::VE, v);
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(cons
   }
   // Ragged last item, by the slice owner's first CTA.
   if (threadIdx.x == 32 && c.b == 0 && full_items < a.items && full_items >= lo && full_items < hi) {
-    const uint4 v = reduce_item<D>(a.ptr, 0, a.P, full_items, a.n);
+    const uint4 v = reduce_item_out<D, kQ8>(a.ptr, 0, a.P, full_items, a.n);
     for (int p = 0; p < a.P; ++p) store_item<D, true>(a.ptr.out[p], full_items, a.n, v);
   }
   if (a.edge_sync) {
@@ -286,8 +289,9 @@ __global__ void __launch_bounds__(32 + kStageItems) k_twostage_write_staged(cons
 //
 // With kScatter the same kernel is the standalone reduce-scatter: rank r's
 // slice is its chunk (n / P elements, a whole number of items) and the result
-// goes to out[r] only, at the chunk's local offset.
-template <class D, int TI, int S, bool kScatter = false>
+// goes to out[r] only, at the chunk's local offset. kQ8: inputs and reduced
+// slice pass the fp8 wire.
+template <class D, int TI, int S, bool kScatter = false, bool kQ8 = false>
 __global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   pdl_trigger();
@@ -332,9 +336,9 @@ __global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
     if (it < hi_full) {
       const unsigned char* src = mine + (k % S) * stage_bytes;
       Acc<D> acc;
-      acc.init(ld_shared_v4(src));
-      for (int p = 1; p < a.P; ++p) acc.add(ld_shared_v4(src + p * (TI * 16)));
-      const uint4 v = acc.round();
+      acc.template init_in<kQ8>(ld_shared_v4(src));
+      for (int p = 1; p < a.P; ++p) acc.template add_in<kQ8>(ld_shared_v4(src + p * (TI * 16)));
+      const uint4 v = acc.template round_out<kQ8>();
       if (kScatter) {
         st_stream(static_cast<typename D::E*>(a.ptr.out[c.r]) + (it - lo) * D::VE, v);
       } else {
@@ -347,7 +351,7 @@ __global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
   }
   cp_async_wait<0>();
   if (!kScatter && threadIdx.x == 0 && c.b == 0 && full_items < a.items && full_items >= lo && full_items < hi) {
-    const uint4 v = reduce_item<D>(a.ptr, 0, a.P, full_items, a.n);
+    const uint4 v = reduce_item_out<D, kQ8>(a.ptr, 0, a.P, full_items, a.n);
     for (int p = 0; p < a.P; ++p) store_item<D, true>(a.ptr.out[p], full_items, a.n, v);
   }
   if (a.edge_sync) {

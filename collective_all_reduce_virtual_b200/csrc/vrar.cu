@@ -28,6 +28,7 @@ struct Settings {
   std::atomic<int> spin_stats{0};
   std::atomic<int> max_ctas{0};  // grid cap per call, 0 = none
   std::atomic<int> payload_wire{VRAR_WIRE_ELEMENT};
+  std::atomic<int> fp8_quant{0};
 };
 Settings g_set;
 
@@ -403,10 +404,15 @@ char shape_choice(int P, size_t bytes) {
 
 // Which write-mode kernel runs a TWOSTAGE_WRITE call. Shapes the table gives
 // to one-shot (when write mode is asked for by name) take the async kernel,
-// the fastest write kernel on small messages.
-int write_kernel_for(int P, size_t bytes) {
+// the fastest write kernel on small messages. With fp8 payloads (q8) the
+// kernels are bound by the quantisation arithmetic, not by memory: the plain
+// kernel's 512-thread CTAs keep the most arithmetic in flight up to 1 MiB per
+// rank, the async kernel above (measured at 8 ranks: 9.5 against 12.2 us at
+// 1 MiB; 18.1, 56 and 185 us against 18.3, 71 and 214 at 2, 8 and 28 MiB).
+int write_kernel_for(int P, size_t bytes, bool q8 = false) {
   const int forced = write_kernel_override();
   if (forced >= 0) return forced;
+  if (q8) return bytes <= (1u << 20) ? kWritePlain : kWriteAsync;
   const char ch = shape_choice(P, bytes);
   return ch == 'P' ? kWritePlain : ch == 'S' ? kWriteStaged : kWriteAsync;
 }
@@ -443,16 +449,28 @@ constexpr int kSmallThreads = 128;
 // mid barrier (measured 6-10 % faster than 512 from 128 KiB to 2 MiB per rank).
 constexpr int kPullThreads = 256;
 
-KernelFn pull_dt(vrar_dtype_t dt) {
-  return dt == VRAR_BF16   ? k_twostage<Bf16T, kPullThreads>
-         : dt == VRAR_FP16 ? k_twostage<F16T, kPullThreads>
-                           : k_twostage<F32T, kPullThreads>;
+// Kernels of the custom all-reduce (one-shot, pull 2-stage, plain write), with
+// or without the fp8 wire (q8, 16-bit element types only; the host rejects
+// fp8 for fp32 before it gets here).
+template <class D>
+KernelFn custom_kernel(vrar_algo_t algo, int threads, bool q8) {
+  if constexpr (D::VE == 8) {
+    if (q8) {
+      if (algo == VRAR_ALGO_ONESHOT)
+        return threads == kSmallThreads ? k_oneshot<D, kSmallThreads, true> : k_oneshot<D, kThreads, true>;
+      if (algo == VRAR_ALGO_TWOSTAGE) return k_twostage<D, kPullThreads, true>;
+      return k_twostage_write<D, true>;
+    }
+  }
+  if (algo == VRAR_ALGO_ONESHOT) return threads == kSmallThreads ? k_oneshot<D, kSmallThreads> : k_oneshot<D>;
+  if (algo == VRAR_ALGO_TWOSTAGE) return k_twostage<D, kPullThreads>;
+  return k_twostage_write<D>;
 }
 
-KernelFn oneshot_small_dt(vrar_dtype_t dt) {
-  return dt == VRAR_BF16   ? k_oneshot<Bf16T, kSmallThreads>
-         : dt == VRAR_FP16 ? k_oneshot<F16T, kSmallThreads>
-                           : k_oneshot<F32T, kSmallThreads>;
+KernelFn custom_kernel_dt(vrar_dtype_t dt, vrar_algo_t algo, int threads, bool q8) {
+  return dt == VRAR_BF16   ? custom_kernel<Bf16T>(algo, threads, q8)
+         : dt == VRAR_FP16 ? custom_kernel<F16T>(algo, threads, q8)
+                           : custom_kernel<F32T>(algo, threads, false);
 }
 
 // HIER (element wire) by size, measured at 4 groups x 8 ranks: up to 256 KiB
@@ -488,25 +506,39 @@ KernelFn async_rs_kernel_dt(vrar_dtype_t dt, int S) {
                                                                      : async_rs_kernel<F32T>(S);
 }
 
-template <class D>
+template <class D, bool Q>
 KernelFn async_kernel(int S) {
   switch (S) {
-    case 8: return k_twostage_write_async<D, kAsyncTileItems, 8>;
-    case 6: return k_twostage_write_async<D, kAsyncTileItems, 6>;
-    case 4: return k_twostage_write_async<D, kAsyncTileItems, 4>;
-    default: return k_twostage_write_async<D, kAsyncTileItems, 3>;
+    case 8: return k_twostage_write_async<D, kAsyncTileItems, 8, false, Q>;
+    case 6: return k_twostage_write_async<D, kAsyncTileItems, 6, false, Q>;
+    case 4: return k_twostage_write_async<D, kAsyncTileItems, 4, false, Q>;
+    default: return k_twostage_write_async<D, kAsyncTileItems, 3, false, Q>;
   }
 }
 
-KernelFn async_kernel_dt(vrar_dtype_t dt, int S) {
-  return dt == VRAR_BF16 ? async_kernel<Bf16T>(S) : dt == VRAR_FP16 ? async_kernel<F16T>(S) : async_kernel<F32T>(S);
+KernelFn async_kernel_dt(vrar_dtype_t dt, int S, bool q8) {
+  if (dt == VRAR_BF16) return q8 ? async_kernel<Bf16T, true>(S) : async_kernel<Bf16T, false>(S);
+  if (dt == VRAR_FP16) return q8 ? async_kernel<F16T, true>(S) : async_kernel<F16T, false>(S);
+  return async_kernel<F32T, false>(S);
 }
 
-constexpr int kWriteTileItems = 64;  // staged write mode: items per tile (1 KiB per input rank)
+// Staged write mode without a CTA budget: items per tile (64: 1 KiB per input
+// rank), the shared-memory bytes of stages a CTA aims for, and the most stages.
+#ifndef VRAR_STAGED_TILE
+#define VRAR_STAGED_TILE 64
+#endif
+#ifndef VRAR_STAGED_BYTES
+#define VRAR_STAGED_BYTES (96 * 1024)
+#endif
+#ifndef VRAR_STAGED_MAX_STAGES
+#define VRAR_STAGED_MAX_STAGES 6
+#endif
+constexpr int kWriteTileItems = VRAR_STAGED_TILE;
+static_assert(kWriteTileItems == 64 || kWriteTileItems == 128, "staged tiles of 64 or 128 items are instantiated");
 
-template <class D>
+template <class D, bool Q>
 KernelFn staged_kernel(int ti) {
-  return ti == 64 ? k_twostage_write_staged<D, 64> : k_twostage_write_staged<D, 128>;
+  return ti == 64 ? k_twostage_write_staged<D, 64, Q> : k_twostage_write_staged<D, 128, Q>;
 }
 
 // Dispatch on the element type.
@@ -515,9 +547,10 @@ KernelFn pick_kernel_dt(vrar_dtype_t dt, vrar_algo_t algo, int C) {
                                                                         : pick_kernel<F32T>(algo, C);
 }
 
-KernelFn staged_kernel_dt(vrar_dtype_t dt, int ti) {
-  return dt == VRAR_BF16 ? staged_kernel<Bf16T>(ti) : dt == VRAR_FP16 ? staged_kernel<F16T>(ti)
-                                                                      : staged_kernel<F32T>(ti);
+KernelFn staged_kernel_dt(vrar_dtype_t dt, int ti, bool q8) {
+  if (dt == VRAR_BF16) return q8 ? staged_kernel<Bf16T, true>(ti) : staged_kernel<Bf16T, false>(ti);
+  if (dt == VRAR_FP16) return q8 ? staged_kernel<F16T, true>(ti) : staged_kernel<F16T, false>(ti);
+  return staged_kernel<F32T, false>(ti);
 }
 
 template <class D>
@@ -558,11 +591,35 @@ struct PayloadPlan {
   size_t bytes = 0;          // slot bytes in all: slot_sets * P * steps * slot_items * 32
 };
 
+// Whether a kernel uses local memory (register spills or a stack frame). The
+// CUDA driver reserves local memory for the whole device the first time it
+// runs a kernel that needs some, which is an allocation the allocation-free
+// entry point avoids by preferring kernels that need none. Cached per kernel.
+bool uses_local_memory(KernelFn fn) {
+  static std::mutex mu;
+  static KernelFn seen[256];
+  static bool local[256];
+  static int used = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (seen[i] == fn) return local[i];
+  cudaFuncAttributes at;
+  bool v = true;
+  if (cudaFuncGetAttributes(&at, fn) == cudaSuccess) v = at.localSizeBytes > 0;
+  else cudaGetLastError();
+  if (used < 256) {
+    seen[used] = fn;
+    local[used++] = v;
+  }
+  return v;
+}
+
 // C_cfg: the configured chunk count. `fit_one_round` (the allocation-free
 // entry point) takes the smallest chunk count up to the kernels' maximum that
 // covers the message in one round, whatever C_cfg is; if none does, at most 4
 // (at most 1 on the fp32 wire), which keeps its two slot sets below the
-// one-round size.
+// one-round size. Among those it skips kernels that use local memory when a
+// larger (or, past one round, smaller) chunk count gives one that uses none.
 int plan_payload(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L, int dev, int sms, int C_cfg,
                  bool fit_one_round, PayloadPlan* out) {
   PayloadPlan pl;
@@ -579,14 +636,24 @@ int plan_payload(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L, int 
   // per rank the element-wire kernel also runs two CTAs per SM (below).
   if (algo == VRAR_ALGO_HIER) C = n * elem_size(dt) <= kHierOnePieceBytes ? 1 : std::min(C, 2);
   if (fit_one_round) {
+    auto kern = [&](int c) { return wide ? pick_wide_dt(dt, algo, c) : pick_kernel_dt(dt, algo, c); };
     const int cmax = wide ? 2 : 8;
-    int pick = 0;
+    int pick = 0, pick_any = 0;
     for (int c = 1; c <= cmax && !pick; ++c) {
-      KernelFn f = wide ? pick_wide_dt(dt, algo, c) : pick_kernel_dt(dt, algo, c);
-      const int cap = std::max(1, std::min(grid_budget(f, dev, sms), kMaxCtas) / P);
-      if ((piece + c - 1) / c <= static_cast<int64_t>(cap) * kThreads) pick = c;
+      const int cap = std::max(1, std::min(grid_budget(kern(c), dev, sms), kMaxCtas) / P);
+      if ((piece + c - 1) / c <= static_cast<int64_t>(cap) * kThreads) {
+        if (!pick_any) pick_any = c;
+        if (!uses_local_memory(kern(c))) pick = c;
+      }
     }
-    C = pick ? pick : (wide ? 1 : std::min(C, 4));
+    if (!pick) pick = pick_any;
+    if (!pick) {  // several rounds: at most 4 pieces (1 on the fp32 wire), preferring no local memory
+      const int top = wide ? 1 : std::min(C, 4);
+      for (int c = top; c >= 1 && !pick; --c)
+        if (!uses_local_memory(kern(c))) pick = c;
+      if (!pick) pick = top;
+    }
+    C = pick;
   } else {
     C = wide ? wide_chunks_for(dt, algo, C, piece, P, dev, sms) : rd_chunks_for_dt(dt, algo, C, piece, P, dev, sms);
   }
@@ -653,6 +720,10 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   }
   const int L = g_set.group_size.load();
   if ((rc = check_shape(algo, P, L)) != VRAR_OK) return rc;
+  // fp8 payloads are defined for the custom all-reduce algorithms on 16-bit
+  // elements (groups of 8 elements = one 16-byte item).
+  const bool q8 = g_set.fp8_quant.load() != 0;
+  if (q8 && (dtype == VRAR_FP32 || algo == VRAR_ALGO_RD || algo == VRAR_ALGO_HIER)) return VRAR_ENOTSUP;
   if (n == 0) return VRAR_OK;
 
   int dev = 0;
@@ -702,12 +773,12 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     case VRAR_ALGO_TWOSTAGE_WRITE: work = (a.items + P - 1) / P; break;
     default: break;
   }
-  const int wk = algo == VRAR_ALGO_TWOSTAGE_WRITE ? write_kernel_for(P, n * elem_size(dtype)) : kWritePlain;
+  const int wk = algo == VRAR_ALGO_TWOSTAGE_WRITE ? write_kernel_for(P, n * elem_size(dtype), q8) : kWritePlain;
   if (wk == kWriteAsync) {
     const int cap_budget = g_set.max_ctas.load();
     const bool deep = cap_budget > 0 && cap_budget <= sms;
     const int S = async_stages(P, n * elem_size(dtype), deep);
-    KernelFn af = async_kernel_dt(dtype, S);
+    KernelFn af = async_kernel_dt(dtype, S, q8);
     const int64_t tiles = std::max<int64_t>(1, (work + kAsyncTileItems - 1) / kAsyncTileItems);
     const size_t smem = static_cast<size_t>(S) * P * kAsyncTileItems * 16;
     const int resident = grid_budget(af, dev, sms, kAsyncTileItems, smem);
@@ -723,9 +794,10 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     const int cap_budget = g_set.max_ctas.load();
     const bool deep = cap_budget > 0 && cap_budget <= sms;
     const int ti = deep ? 128 : kWriteTileItems;
-    KernelFn sf = staged_kernel_dt(dtype, ti);
+    KernelFn sf = staged_kernel_dt(dtype, ti, q8);
     const int64_t tiles = std::max<int64_t>(1, (work + ti - 1) / ti);
-    const int S = std::max(2, std::min(deep ? kMaxStages : 6, ((deep ? 192 : 96) * 1024) / (P * ti * 16)));
+    const int S = std::max(2, std::min(deep ? kMaxStages : VRAR_STAGED_MAX_STAGES,
+                                       (deep ? 192 * 1024 : VRAR_STAGED_BYTES) / (P * ti * 16)));
     const size_t smem = kStagedHeader + static_cast<size_t>(S) * P * ti * 16;
     const int resident = grid_budget(sf, dev, sms, 32 + ti, smem);
     const int B = static_cast<int>(std::min<int64_t>(tiles, std::max(1, std::min(resident, kMaxCtas) / P)));
@@ -735,14 +807,10 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     return launch(sf, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), 32 + ti, smem);
   }
   int threads = kThreads;
-  if (algo == VRAR_ALGO_ONESHOT && static_cast<size_t>(P) * n * elem_size(dtype) <= kOneshotSmallBytes) {
-    fn = oneshot_small_dt(dtype);
+  if (algo == VRAR_ALGO_ONESHOT && static_cast<size_t>(P) * n * elem_size(dtype) <= kOneshotSmallBytes)
     threads = kSmallThreads;
-  }
-  if (algo == VRAR_ALGO_TWOSTAGE) {
-    fn = pull_dt(dtype);
-    threads = kPullThreads;
-  }
+  if (algo == VRAR_ALGO_TWOSTAGE) threads = kPullThreads;
+  fn = custom_kernel_dt(dtype, algo, threads, q8);
   a.B = blocks_per_rank(work, P, grid_budget(fn, dev, sms, threads), threads);
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), threads);
 }
@@ -844,7 +912,7 @@ const char* vrar_kernel_name(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t al
     case VRAR_ALGO_ONESHOT: return "k_oneshot";
     case VRAR_ALGO_TWOSTAGE: return "k_twostage";
     case VRAR_ALGO_TWOSTAGE_WRITE: {
-      const int wk = write_kernel_for(P, n * elem_size(dtype));
+      const int wk = write_kernel_for(P, n * elem_size(dtype), g_set.fp8_quant.load() != 0 && dtype != VRAR_FP32);
       return wk == kWriteAsync ? "k_twostage_write_async" : wk == kWriteStaged ? "k_twostage_write_staged"
                                                                                 : "k_twostage_write";
     }
@@ -969,6 +1037,12 @@ int vrar_set_payload_wire(int wire) {
   return VRAR_OK;
 }
 int vrar_get_payload_wire(void) { return g_set.payload_wire.load(); }
+
+int vrar_set_fp8_quant(int on) {
+  g_set.fp8_quant = on ? 1 : 0;
+  return VRAR_OK;
+}
+int vrar_get_fp8_quant(void) { return g_set.fp8_quant.load(); }
 
 int vrar_set_spin_stats(int on) {
   g_set.spin_stats = on ? 1 : 0;

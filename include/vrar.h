@@ -158,7 +158,8 @@ VRAR_API int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype);
  * "k_twostage_write" (plain), "k_twostage_write_staged" (bulk copies into
  * shared memory by one producer lane), "k_twostage_write_async" (per-thread
  * async copies into shared memory), chosen per shape from the same measured
- * table as vrar_select_algo. For profilers and benchmarks; the sources have
+ * table as vrar_select_algo (with fp8 payloads on: the plain kernel up to 1 MiB per
+ * rank, the async kernel above). For profilers and benchmarks; the sources have
  * no counterpart. Returns a static string, or NULL for invalid arguments
  * (P outside 1..VRAR_MAX_RANKS, unknown dtype or algorithm). Launches nothing.
  */
@@ -190,6 +191,33 @@ VRAR_API int vrar_get_rd_chunks(void);
 enum { VRAR_WIRE_ELEMENT = 0, VRAR_WIRE_FP32 = 1 };
 VRAR_API int vrar_set_payload_wire(int wire);
 VRAR_API int vrar_get_payload_wire(void);
+
+/* fp8 payloads of the custom all-reduce: the ca_fp8_quant flag that the
+ * ROCm/ATOM pull request 1681 page passes at the RowParallelLinear all-reduce
+ * call site ("all_reduce(y, ca_fp8_quant=False)"). The page names the flag and
+ * nothing more, so the scheme is this library's reading: with the setting on,
+ * every value that passes from one rank to another in ONESHOT, TWOSTAGE and
+ * TWOSTAGE_WRITE (and AUTO, which picks among them) travels as OCP FP8 E4M3
+ * (4 exponent bits biased by 7, 3 fraction bits, subnormals kept, no
+ * infinities, largest finite 448) with one binary32 scale per group of 8
+ * elements (one 16-byte item of a bf16 / fp16 vector): s = amax / 448 (amax =
+ * the group's largest magnitude; s = 1 when that gives 0), q = E4M3(x / s)
+ * rounded to nearest even and saturated at 448, received as q * s (binary32
+ * division and product, round to nearest even). ONESHOT passes every input
+ * through it once (each rank's own input too, so all outputs agree):
+ *   y = rnd_T(fp8(x_0) + fp8(x_1) + ... + fp8(x_{P-1}))   (binary32 adds, in order)
+ * TWOSTAGE and TWOSTAGE_WRITE pass the inputs through it for the
+ * reduce-scatter and the reduced binary32 slice again for the all-gather:
+ *   y = rnd_T(fp8(fp8(x_0) + ... + fp8(x_{P-1})))
+ * On one device nothing is stored in fp8: the kernels quantise and dequantise
+ * in registers where a value would cross between ranks, so a call moves the
+ * same bytes as without it. Inputs must be finite; a group whose binary32
+ * sum overflows to infinity has an infinite scale in the 2-stage's second
+ * quantisation and comes back as NaN. With the setting on, fp32 elements, RD
+ * and HIER return VRAR_ENOTSUP. Default 0 (off). Process-wide setting, read
+ * when a call is queued. */
+VRAR_API int vrar_set_fp8_quant(int on);
+VRAR_API int vrar_get_fp8_quant(void);
 
 /* Whether ONESHOT / TWOSTAGE / TWOSTAGE_WRITE run the start and end flag
  * barriers of [CAR] (default 0 = no). Across devices they keep a rank from
@@ -290,6 +318,16 @@ VRAR_API int vrar_debug_set_fault_mask(uint32_t mask);
  *    call waits for carries that call's sequence number. Calls that overlap on
  *    the GPU (on different streams, or from several host threads) race on the
  *    array and give wrong results: keep them ordered on one stream.
+ *  - The CUDA driver can reserve device memory behind any kernel launch, which
+ *    this call cannot prevent: with lazy module loading (the default since
+ *    CUDA 12.2) it loads a kernel's code the first time that kernel is used,
+ *    and it reserves local memory for the whole device the first time it runs
+ *    a kernel that needs local memory. This call picks, among the kernel
+ *    variants that suit the request, one that uses no local memory (asked of
+ *    the runtime with cudaFuncGetAttributes); with CUDA_MODULE_LOADING=EAGER
+ *    in the environment all of the library's code is loaded when the library
+ *    first calls the CUDA runtime, and a call then changes the device's free
+ *    memory by nothing.
  *  - Device waits are bounded as in every other call (vrar_set_spin_timeout_ns)
  *    and honour vrar_debug_set_fault_mask. A wait that runs out of time
  *    records VRAR_ETIMEDOUT in the array's status word, and the outputs of the

@@ -57,7 +57,8 @@
  *    agree); the 2-stage variants quantise the inputs for the reduce-scatter
  *    and the reduced binary32 slice again for the all-gather, and every rank,
  *    the owner included, stores the dequantised value rounded to the tensor
- *    type.
+ *    type. A group whose binary32 sum is infinite has an infinite scale in
+ *    that second quantisation, so all its values come back as NaN.
  *
  * Floating-point environment: the functions below clear the x86 flush-to-zero
  * and denormals-are-zero bits for their duration, so subnormal inputs and
