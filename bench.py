@@ -825,7 +825,8 @@ def run_selector_sweep(args):
 
 def run_case(spec_text: str):
     """A few back-to-back calls of one algorithm on one shape (for profilers):
-    'algo,P,KiB[,calls]', algo an all-reduce algorithm or 'rs' / 'ag' (the
+    'algo,P,KiB[,calls]', algo an all-reduce algorithm (with '+edge' and / or
+    '+fp8' for the start/end barriers and the fp8 payloads) or 'rs' / 'ag' (the
     standalone reduce-scatter / all-gather; KiB is the full per-rank vector).
     Exits non-zero if the device status is not clean."""
     import collective_all_reduce_virtual_b200 as vrar
@@ -836,12 +837,13 @@ def run_case(spec_text: str):
     torch.cuda.set_device(device)
     wl = Workload(dict(DECODE, P=P, n=kib * 512, name=spec_text), device)
     h = torch.cuda.current_stream().cuda_stream
-    for i in range(calls):
-        if algo in ("rs", "ag"):
-            wl.collective_call(i, algo, h)
-        else:
-            wl.call(i, algo, h)
-    torch.cuda.synchronize()
+    with flags_set(vrar, algo) as base:
+        for i in range(calls):
+            if base in ("rs", "ag"):
+                wl.collective_call(i, base, h)
+            else:
+                wl.call(i, base, h)
+        torch.cuda.synchronize()
     rc, info = vrar.query_status()
     print(json.dumps({"case": spec_text, "status": rc, "info": info}))
     return rc

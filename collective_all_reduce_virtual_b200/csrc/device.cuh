@@ -144,13 +144,18 @@ __device__ __forceinline__ void st_stream(void* p, uint4 v) {
                : "memory");
 }
 
-// Two fused payload words; each 8-byte element is one single-copy-atomic access.
-__device__ __forceinline__ void st_payload2(uint64_t* p, uint64_t a, uint64_t b) {
-  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1,%2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+// Four fused payload words (one 32-byte slot, 32-byte aligned) in one 256-bit
+// access, which sm_100 has for global memory. A vector access is performed as
+// accesses of its 8-byte elements, each single-copy atomic, in no fixed order:
+// the reader still checks the tag of every word.
+__device__ __forceinline__ void st_payload4(uint64_t* p, uint64_t a, uint64_t b, uint64_t c, uint64_t d) {
+  asm volatile("st.relaxed.gpu.global.v4.u64 [%0], {%1,%2,%3,%4};" ::"l"(p), "l"(a), "l"(b), "l"(c), "l"(d)
+               : "memory");
 }
 
-__device__ __forceinline__ void ld_payload2(const uint64_t* p, uint64_t& a, uint64_t& b) {
-  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0,%1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+__device__ __forceinline__ void ld_payload4(const uint64_t* p, uint64_t& a, uint64_t& b, uint64_t& c, uint64_t& d) {
+  asm volatile("ld.relaxed.gpu.global.v4.u64 {%0,%1,%2,%3}, [%4];" : "=l"(a), "=l"(b), "=l"(c), "=l"(d) : "l"(p)
+               : "memory");
 }
 
 // ---- shared-memory pipelines: mbarriers and bulk copies (no multicast) -------------------
@@ -660,8 +665,7 @@ __device__ __forceinline__ bool block_barrier(const KArgs& a, const Cta& c, uint
 
 __device__ __forceinline__ void send_item(uint64_t* slot, const uint4& v, uint32_t flag) {
   const uint64_t hi = static_cast<uint64_t>(flag) << 32;
-  st_payload2(slot, hi | v.x, hi | v.y);
-  st_payload2(slot + 2, hi | v.z, hi | v.w);
+  st_payload4(slot, hi | v.x, hi | v.y, hi | v.z, hi | v.w);
 }
 
 }  // namespace vrar

@@ -427,8 +427,7 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       if (val[k]) {
-        ld_payload2(src + slot[k] * 4, w[k][0], w[k][1]);
-        ld_payload2(src + slot[k] * 4 + 2, w[k][2], w[k][3]);
+        ld_payload4(src + slot[k] * 4, w[k][0], w[k][1], w[k][2], w[k][3]);
         pending |= 1u << k;
       }
     }
@@ -454,12 +453,8 @@ __device__ __forceinline__ bool rd_exchange(const KArgs& a, const Cta& c, uint4 
         }
       }
 #pragma unroll
-      for (int k = 0; k < C; ++k) {
-        if ((pending >> k) & 1u) {
-          ld_payload2(src + slot[k] * 4, w[k][0], w[k][1]);
-          ld_payload2(src + slot[k] * 4 + 2, w[k][2], w[k][3]);
-        }
-      }
+      for (int k = 0; k < C; ++k)
+        if ((pending >> k) & 1u) ld_payload4(src + slot[k] * 4, w[k][0], w[k][1], w[k][2], w[k][3]);
     }
     if (val[0]) record_spins(a, it + 1, false);  // one wait per step (the C pieces are polled together)
 #pragma unroll
@@ -488,8 +483,11 @@ __device__ __forceinline__ void prefetch_next_round(const void* in, int64_t lo, 
   }
 }
 
-template <class D, int C>
-__global__ void __launch_bounds__(kThreads) k_rd(const KArgs a) {
+// kMinBlocks 2 limits registers to fit two CTAs per SM (64 per thread: at most
+// two pieces per thread without spills), which the library launches for the
+// element wire (more threads in flight per SM; measured faster).
+template <class D, int C, int kMinBlocks = 1>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) k_rd(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;

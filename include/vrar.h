@@ -174,9 +174,11 @@ VRAR_API int vrar_get_group_size(void);
  * cut into chunks and every thread keeps up to C payload pieces, one per chunk,
  * in flight per step ([NVRAR] "Chunked Non-blocking Communication"). A call
  * uses fewer than C when its grid has threads to spare for a short message.
- * VRAR_ALGO_HIER uses at most 2, and 1 up to 2 MiB per rank (measured
- * faster: its in-group phases keep L loads and stores per piece in flight
- * already).
+ * VRAR_ALGO_RD on the element wire uses at most 2 (its kernel runs two CTAs
+ * per SM with 64 registers per thread, measured faster than one CTA with more
+ * pieces); VRAR_ALGO_HIER uses at most 2, and 1 up to 2 MiB per rank
+ * (measured faster: its in-group phases keep L loads and stores per piece in
+ * flight already); the fp32 wire at most 2; vrar_allreduce_rd_noalloc up to 8.
  * Results do not depend on C. Range 1..8. */
 VRAR_API int vrar_set_rd_chunks(int C);
 VRAR_API int vrar_get_rd_chunks(void);

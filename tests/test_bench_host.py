@@ -114,3 +114,35 @@ def test_reference_arm_line_on_cpu(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["metric"] == bench.METRIC
+
+
+def test_row_flags():
+    assert bench.with_flags("twostage_write") == ("twostage_write", False, False)
+    assert bench.with_flags("oneshot+edge") == ("oneshot", True, False)
+    assert bench.with_flags("twostage_write+fp8") == ("twostage_write", False, True)
+    assert bench.with_flags("twostage+edge+fp8") == ("twostage", True, True)
+
+
+def test_cpu_baseline_host_facts_and_pinning():
+    import os
+    h = bench.host_description()
+    assert h["nproc"] == os.cpu_count() and h["nproc"] >= 1
+    before = os.sched_getaffinity(0)
+    with bench.one_core() as pin:
+        inside = os.sched_getaffinity(0)
+        assert len(inside) == 1 and inside <= before
+        assert pin.describe() == f"os.sched_setaffinity to core {min(before)}"
+    assert os.sched_getaffinity(0) == before, "the affinity must be restored"
+
+
+def test_reference_arm_prints_one_line_on_the_cpu(capsys):
+    """The reference arm times the CPU oracle on slices of the step's workload
+    and needs no GPU."""
+    import json
+    bench.main(["--impl", "reference", "--steps", "2", "--warmup", "3"])
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["value"] > 0
+    assert line["config"]["workload"] == bench.WORKLOAD["name"] and line["config"]["n"] == 16384 * 7168
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["threads"] == 1 and "nproc" in cb
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0

@@ -543,3 +543,52 @@ def test_payload_slots_are_bounded_by_the_grid():
         assert_bits([to_np(o[lo:lo + 8192]) for o in outs], want, f"rd prefill window {lo}")
     del outs, d_in
     torch.cuda.empty_cache()
+
+
+def test_waits_on_peers_that_cannot_become_resident_end_in_a_timeout():
+    """The waits assume that all CTAs of a call are resident together. When
+    concurrent work holds SMs, that may not hold: then the waits must end with
+    VRAR_ETIMEDOUT, and no output element may ever receive a wrong value. The
+    blocker is the allocation-free entry point (its own control words and
+    slots, so the two calls share no protocol state) with a CTA budget of 72
+    and a rank that never sends: its CTAs hold 72 SMs for its 300 ms limit.
+    Meanwhile a full-grid RD call with a 50 ms limit runs on another stream, on
+    outputs filled with NaN: every element must end either exact or unwritten
+    (a wait that gives up stores nothing), and the status must say a wait ran
+    out."""
+    P, n = 8, 100_003
+    xs = gen(P, n, "bf16", synth.normal(0.0, 1.0), seed=44)
+    want = oracle.allreduce("rd", xs, "bf16")
+    d_in = _dev(xs, "bf16")
+    outs = [torch.empty_like(t) for t in d_in]
+    blk_out = [torch.empty_like(t) for t in d_in]
+    vrar.all_reduce(d_in, outs, algo="rd")  # sizes the workspace
+    for t in outs:
+        t.fill_(float("nan"))
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    lib = vrar.lib()
+    vrar.set_max_ctas(72)
+    vrar.set_spin_timeout_ns(300_000_000)
+    vrar.debug_set_fault_mask(1 << 3)
+    rc = lib.vrar_allreduce_rd_noalloc(vrar.ptr_array([t.data_ptr() for t in d_in]),
+                                       vrar.ptr_array([t.data_ptr() for t in blk_out]), P, n, 0, s1.cuda_stream)
+    assert rc == vrar.OK
+    vrar.set_max_ctas(0)
+    vrar.debug_set_fault_mask(0)
+    vrar.set_spin_timeout_ns(50_000_000)
+    vrar.all_reduce(d_in, outs, algo="rd", stream=s2)
+    torch.cuda.synchronize()
+    rc, info = vrar.query_status()
+    assert rc == vrar.ETIMEDOUT, (rc, info)
+    unwritten = 0
+    for p in range(P):
+        got = to_np(outs[p])
+        nan = np.isnan(oracle.to_float(got, "bf16"))
+        unwritten += int(nan.sum())
+        assert (got[~nan] == want[p][~nan]).all(), f"rank {p}: a written element is wrong"
+    print(f"elements left unwritten by the contended call: {unwritten} of {P * n}")
+    # Alone again, the same call is exact.
+    outs = vrar.all_reduce(d_in, algo="rd")
+    assert vrar.query_status()[0] == 0
+    assert_bits([to_np(o) for o in outs], want, "rd after the contention")
