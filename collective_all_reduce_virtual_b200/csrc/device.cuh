@@ -76,6 +76,7 @@ struct KArgs {
   uint64_t* ll;      // payload slots
   int64_t slot_items;  // payload slots (32 bytes each) per rank, step and slot set
   int slot_sets;       // 1: slot = item index (one round); 2: slots reused by round parity
+  int prefetch_next;   // hierarchical: warm L2 with the next round's inputs
   unsigned long long* stats;  // spin statistics, or null when they are off
 };
 

@@ -573,6 +573,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_hier(const KArgs a) {
     }
     if (base == 0) cta_publish_flag(c, ticket);
     if (!ok) continue;
+    // The next round reads the same items of all L inputs of the group: warm
+    // L2 with them while this round's exchange runs (threads 0..L*C-1, one
+    // input and chunk each), when the host asks for it (prefetch_next).
+    if (a.prefetch_next && threadIdx.x < L * C) {
+      const int64_t k = threadIdx.x % C;
+      const int64_t first = base + stride + static_cast<int64_t>(c.b) * kThreads;
+      const int64_t end = min((k + 1) * per_chunk, len) - k * per_chunk;
+      if (first < end)
+        prefetch_items<D>(a.ptr.in[g * L + threadIdx.x / C], lo + k * per_chunk + first,
+                          min(static_cast<int64_t>(kThreads), end - first), a.n);
+    }
     ok = rd_exchange<D, C, true>(a, c, v, slot, val, a.slot_sets == 1 ? 0 : static_cast<int>(rnd & 1),
                                  rd_tag(c.flag, rnd));
     if (ok) {
@@ -594,9 +605,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_hier(const KArgs a) {
 // twice the payload words of the element-type wire); the steps add in fp32
 // without rounding, and the store rounds once to the element type. A slot of
 // the element wire becomes two quad slots (2 * slot, 2 * slot + 1); the host
-// doubles slot_items. C is at most 2 here (2C quads in flight per thread).
-template <class D, int C>
-__global__ void __launch_bounds__(kThreads) k_rd_wide(const KArgs a) {
+// doubles slot_items. C is at most 2 here (2C quads in flight per thread); the
+// library runs k_rd_wide with one piece and two CTAs per SM (kMinBlocks 2).
+template <class D, int C, int kMinBlocks = 1>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) k_rd_wide(const KArgs a) {
   pdl_trigger();
   Cta c = cta_coords(a);
   const int64_t stride = static_cast<int64_t>(a.B) * kThreads;

@@ -380,18 +380,19 @@ int write_kernel_override() {
 // the bulk-copy staged kernel, 'P' write mode with the plain kernel. Rows:
 // P <= 2, 4, 8, 16, 32; columns: bytes per rank <= 32 KiB, 64 KiB, ...,
 // 8 MiB, and above. One-shot keeps small messages at two and four ranks (one
-// pass, its re-reads served by L2). The async write kernel wins almost everywhere
-// else: every thread keeps all P loads of its items in flight, with no
-// serial issue. From 8 MiB per rank at 4-16 ranks the bulk-copy pipeline
-// streams a little better, and at 32 ranks from 4 MiB the plain kernel
-// (shared-memory stages of 32 ranks cost occupancy); both margins are a few
-// percent.
+// pass, its re-reads served by L2); at two ranks and 2 MiB per rank the plain
+// write kernel is faster (2.70 against 3.19 us). The async write kernel wins
+// almost everywhere else: every thread keeps all P loads of its items in
+// flight, with no serial issue. From 8 MiB per rank at 4-16 ranks the
+// bulk-copy pipeline streams a little better, and at 32 ranks at 4 and 8 MiB
+// the plain kernel (shared-memory stages of 32 ranks cost occupancy); those
+// margins are a few percent.
 constexpr char kChoice[5][10] = {
-    {'O', 'O', 'O', 'O', 'O', 'O', 'O', 'A', 'A', 'A'},  // P <= 2
+    {'O', 'O', 'O', 'O', 'O', 'O', 'P', 'A', 'A', 'A'},  // P <= 2
     {'O', 'O', 'A', 'O', 'O', 'A', 'A', 'A', 'S', 'A'},  // P <= 4
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 8
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 16
-    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'P'},  // P <= 32
+    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'A'},  // P <= 32
 };
 
 char shape_choice(int P, size_t bytes) {
@@ -481,6 +482,12 @@ KernelFn custom_kernel_dt(vrar_dtype_t dt, vrar_algo_t algo, int threads, bool q
 constexpr size_t kHierOneCtaBytes = 256 << 10;
 constexpr size_t kHierOnePieceBytes = 2 << 20;
 
+// HIER warms L2 with each next round's group inputs up to 2 MiB per rank
+// (measured: 18.7 against 20.1 us at 4 x 8 ranks x 1 MiB, 16.3 against 17.8 at
+// 2 x 8 x 2 MiB, 20.5 against 22.2 at 4 x 2 x 2 MiB); above it the early loads
+// evict payload slots (209 against 177 us at 4 x 8 x 8 MiB).
+constexpr size_t kHierPrefetchBytes = 2 << 20;
+
 template <class D>
 KernelFn hier_two_per_sm(int C) {
   return C <= 1 ? k_hier<D, 1, 2> : k_hier<D, 2, 2>;
@@ -569,9 +576,14 @@ KernelFn staged_kernel_dt(vrar_dtype_t dt, int ti, bool q8) {
   return staged_kernel<F32T, false>(ti);
 }
 
+// fp32 partials on the wire. RD runs two CTAs per SM with one piece per thread
+// (measured at 8 ranks: 30.6 / 51.6 / 196 us at 1 / 2 / 8 MiB per rank against
+// 31.4 / 57.6 / 205 us with one CTA per SM and two pieces; two pieces in the
+// two-CTA build spill). HIER keeps one CTA per SM (47.0 against 57.8 us at
+// 4 x 8 ranks x 2 MiB with two).
 template <class D>
 KernelFn pick_wide(vrar_algo_t algo, int C) {
-  if (algo == VRAR_ALGO_RD) return C <= 1 ? k_rd_wide<D, 1> : k_rd_wide<D, 2>;
+  if (algo == VRAR_ALGO_RD) return k_rd_wide<D, 1, 2>;
   return C <= 1 ? k_hier_wide<D, 1> : k_hier_wide<D, 2>;
 }
 
@@ -579,10 +591,10 @@ KernelFn pick_wide_dt(vrar_dtype_t dt, vrar_algo_t algo, int C) {
   return dt == VRAR_BF16 ? pick_wide<Bf16T>(algo, C) : pick_wide<F16T>(algo, C);
 }
 
-// Chunk count for the fp32-wire kernels (at most 2, see k_rd_wide), chosen
-// like rd_chunks_for.
+// Chunk count for the fp32-wire kernels (at most 2, see k_rd_wide; RD takes 1,
+// see pick_wide), chosen like rd_chunks_for.
 int wide_chunks_for(vrar_dtype_t dt, vrar_algo_t algo, int C, int64_t work, int P, int dev, int sms) {
-  C = std::min(C, 2);
+  C = algo == VRAR_ALGO_RD ? 1 : std::min(C, 2);
   for (int c = 1; c < C; ++c) {
     const int cap = std::max(1, std::min(grid_budget(pick_wide_dt(dt, algo, c), dev, sms), kMaxCtas) / P);
     if ((work + c - 1) / c <= static_cast<int64_t>(cap) * kThreads) return c;
@@ -633,9 +645,10 @@ bool uses_local_memory(KernelFn fn) {
 // C_cfg: the configured chunk count. `fit_one_round` (the allocation-free
 // entry point) takes the smallest chunk count up to the kernels' maximum that
 // covers the message in one round, whatever C_cfg is; if none does, at most 4
-// (at most 1 on the fp32 wire), which keeps its two slot sets below the
-// one-round size. Among those it skips kernels that use local memory when a
-// larger (or, past one round, smaller) chunk count gives one that uses none.
+// (at most 1 on the fp32 wire), and few enough CTAs per rank that its two slot
+// sets stay within the one-round size. Among those it skips kernels that use
+// local memory when a larger (or, past one round, smaller) chunk count gives
+// one that uses none.
 int plan_payload(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L, int dev, int sms, int C_cfg,
                  bool fit_one_round, PayloadPlan* out) {
   PayloadPlan pl;
@@ -653,7 +666,7 @@ int plan_payload(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L, int 
   if (algo == VRAR_ALGO_HIER) C = n * elem_size(dt) <= kHierOnePieceBytes ? 1 : std::min(C, 2);
   if (fit_one_round) {
     auto kern = [&](int c) { return wide ? pick_wide_dt(dt, algo, c) : pick_kernel_dt(dt, algo, c); };
-    const int cmax = wide ? 2 : 8;
+    const int cmax = wide ? (algo == VRAR_ALGO_RD ? 1 : 2) : 8;  // the kernels' largest chunk count
     int pick = 0, pick_any = 0;
     for (int c = 1; c <= cmax && !pick; ++c) {
       const int cap = std::max(1, std::min(grid_budget(kern(c), dev, sms), kMaxCtas) / P);
@@ -686,6 +699,13 @@ int plan_payload(vrar_algo_t algo, int P, size_t n, vrar_dtype_t dt, int L, int 
   if (!pl.fn) return VRAR_EINVAL;
   const int64_t per_chunk = (piece + C - 1) / C;
   pl.B = blocks_per_rank(per_chunk, P, grid_budget(pl.fn, dev, sms));
+  if (fit_one_round && per_chunk > static_cast<int64_t>(pl.B) * kThreads) {
+    // Several rounds: two slot sets of C * B * T slots each. Keep them within
+    // the one-round size (piece slots), which is what the caller's limit is
+    // stated in: B <= piece / (2 C T).
+    const int64_t cap_b = std::max<int64_t>(1, piece / (2 * static_cast<int64_t>(C) * kThreads));
+    if (pl.B > cap_b) pl.B = static_cast<int>(cap_b);
+  }
   const int64_t stride = static_cast<int64_t>(pl.B) * kThreads;
   const int64_t rounds = (per_chunk + stride - 1) / stride;
   pl.slot_sets = rounds > 1 ? 2 : 1;
@@ -786,6 +806,7 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   if (payload) {
     a.steps = algo == VRAR_ALGO_RD ? ilog2(P) : ilog2(P / L);
     a.B = plan.B;
+    a.prefetch_next = algo == VRAR_ALGO_HIER && n * elem_size(dtype) <= kHierPrefetchBytes;
     return launch(plan.fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream));
   }
 

@@ -147,7 +147,10 @@ def test_selector_table_entries():
     """A few entries of the measured per-shape table (bytes per rank)."""
     bf = torch.bfloat16
     assert vrar.select_algo(1, 1 << 20, bf) == "oneshot"            # a copy
-    assert vrar.select_algo(2, 1 << 20, bf) == "oneshot"            # 2 MiB at 2 ranks
+    assert vrar.select_algo(2, 1 << 19, bf) == "oneshot"            # 1 MiB at 2 ranks
+    assert vrar.select_algo(2, 1 << 20, bf) == "twostage_write"     # 2 MiB at 2 ranks (plain write kernel)
+    assert vrar.kernel_name(2, 1 << 20, bf, "auto") == "k_twostage_write"
+    assert vrar.kernel_name(32, 8 << 20, bf, "auto") == "k_twostage_write_async"  # 16 MiB at 32 ranks
     assert vrar.select_algo(2, 4 << 20, bf) == "twostage_write"     # 8 MiB at 2 ranks
     assert vrar.select_algo(8, 524288, bf) == "twostage_write"      # 1 MiB at 8 ranks (the decode shape)
     assert vrar.select_algo(8, 117440512, bf) == "twostage_write"   # prefill

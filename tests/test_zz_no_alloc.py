@@ -55,12 +55,14 @@ def _noalloc(d_in, outs, P, n, dtype, stream=None):
 # (256 + 8 * 3 * ceil(n / e) * 32 * w <= 16 MiB: n <= 174,760 bf16, 87,380
 # fp32, 87,376 bf16 with fp32 partials on the wire), and calls whose CTA budget
 # makes the grid too small for one round, so that the slots are reused round
-# by round.
+# by round; and 2 ranks with fp32 partials at the limit (256 + 2 * 1 * 131,070
+# * 64 bytes), which needs several rounds.
 CASES = [(4, 7, "bf16", "element", 0), (2, 65_536, "bf16", "element", 0), (8, 100_003, "bf16", "element", 0),
          (8, 174_760, "bf16", "element", 0), (4, 7, "fp32", "element", 0), (2, 65_536, "fp32", "element", 0),
          (8, 50_003, "fp32", "element", 0), (8, 87_380, "fp32", "element", 0), (8, 50_001, "fp16", "element", 0),
          (8, 87_376, "bf16", "fp32", 0),
-         (8, 100_003, "bf16", "element", 16), (16, 60_001, "fp16", "element", 16), (8, 87_376, "bf16", "fp32", 16)]
+         (8, 100_003, "bf16", "element", 16), (16, 60_001, "fp16", "element", 16), (8, 87_376, "bf16", "fp32", 16),
+         (2, 1_048_560, "bf16", "fp32", 0)]  # several rounds at the limit: both slot sets within it
 
 
 @pytest.mark.parametrize("P,n,dtype,wire,budget", CASES)
@@ -92,7 +94,8 @@ def test_noalloc_matches_oracle_and_allocating_rd_on_two_calls(P, n, dtype, wire
 
 
 @pytest.mark.parametrize("P,n,dtype,wire", [(8, 174_761, "bf16", "element"), (8, 87_381, "fp32", "element"),
-                                            (8, 87_377, "bf16", "fp32"), (32, 26_209, "fp16", "element")])
+                                            (8, 87_377, "bf16", "fp32"), (32, 26_209, "fp16", "element"),
+                                            (2, 1_048_561, "bf16", "fp32")])
 def test_noalloc_rejects_one_past_the_limit_and_queues_nothing(P, n, dtype, wire):
     """One element past the limit (for 32 ranks: 256 + 32 * 5 * 3277 * 32 > 16 MiB)
     is refused before anything is queued: the outputs keep their contents."""
