@@ -453,6 +453,25 @@ __device__ __forceinline__ void store_item(void* base, int64_t it, int64_t n, co
     if (i < nv) p[i] = t.e[i];
 }
 
+// Item `it` stored to `count` outputs rank_out[first + (start + j) mod count]
+// for j = 0 .. count-1 (streaming stores): the full-item check is made once.
+template <class D>
+__device__ __forceinline__ void store_item_rotated(void* const* out, int first, int count, int start, int64_t it,
+                                                   int64_t n, const uint4& v) {
+  if ((it + 1) * D::VE <= n) {
+    int q = start;
+    for (int j = 0; j < count; ++j) {
+      st_stream(static_cast<typename D::E*>(out[first + q]) + it * D::VE, v);
+      q = q + 1 == count ? 0 : q + 1;
+    }
+    return;
+  }
+  for (int j = 0; j < count; ++j) {
+    const int q = start + j >= count ? start + j - count : start + j;
+    store_item<D, true>(out[first + q], it, n, v);
+  }
+}
+
 // Ascending-rank fp32 sum of item `it` over ranks first .. first+count-1 (not
 // rounded), each input through the fp8 wire when kQ8. Loads are issued eight
 // at a time so that they overlap; the adds stay in rank order.

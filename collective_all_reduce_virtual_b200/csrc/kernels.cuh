@@ -23,6 +23,14 @@ __device__ __forceinline__ int64_t lo_of(int64_t part, int64_t piece, int64_t to
   return v < total ? v : total;
 }
 
+// (a + b) mod m for 0 <= a, b < m, without an integer division: the rotated
+// rank orders below (stores and peer reads staggered by the rank's own index,
+// so that the ranks do not all touch one buffer at once) are computed per item.
+__device__ __forceinline__ int add_mod(int a, int b, int m) {
+  const int v = a + b;
+  return v >= m ? v - m : v;
+}
+
 // One-shot [CAR, the 1-stage kernel]: every rank reads all P inputs and
 // reduces the whole vector into its own output, between start and end
 // barriers. The P CTAs with the same b read the same items at about the same
@@ -89,7 +97,7 @@ __global__ void __launch_bounds__(T) k_twostage(const KArgs a) {
       int64_t it[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int s = (c.r + j0 + j) % a.P;
+        const int s = add_mod(c.r, j0 + j < a.P ? j0 + j : 0, a.P);  // lanes past P are skipped below
         it[j] = s * piece + off;
         if (j0 + j < a.P && it[j] < lo_of(s + 1, piece, a.items)) v[j] = load_item_peer<D>(a.ptr.out[s], it[j], a.n);
         else it[j] = -1;
@@ -125,11 +133,7 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
   const int64_t piece = (a.items + a.P - 1) / a.P;
   const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
   for (int64_t it = lo + static_cast<int64_t>(c.b) * kThreads + threadIdx.x; it < hi; it += stride) {
-    const uint4 v = reduce_item_out<D, kQ8>(a.ptr, 0, a.P, it, a.n);
-    for (int j = 0; j < a.P; ++j) {
-      const int p = (c.r + j) % a.P;
-      store_item<D, true>(a.ptr.out[p], it, a.n, v);
-    }
+    store_item_rotated<D>(a.ptr.out, 0, a.P, c.r, it, a.n, reduce_item_out<D, kQ8>(a.ptr, 0, a.P, it, a.n));
   }
   if (a.edge_sync) {
     __threadfence();
@@ -343,7 +347,7 @@ __global__ void __launch_bounds__(TI) k_twostage_write_async(const KArgs a) {
         st_stream(static_cast<typename D::E*>(a.ptr.out[c.r]) + (it - lo) * D::VE, v);
       } else {
         for (int j = 0; j < a.P; ++j) {
-          const int q = (c.r + j) % a.P;
+          const int q = add_mod(c.r, j, a.P);
           st_stream(static_cast<typename D::E*>(a.ptr.out[q]) + it * D::VE, v);
         }
       }
@@ -588,13 +592,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_hier(const KArgs a) {
                                  rd_tag(c.flag, rnd));
     if (ok) {
 #pragma unroll
-      for (int k = 0; k < C; ++k) {
-        if (!val[k]) continue;
-        for (int jj = 0; jj < L; ++jj) {
-          const int lp = (l + jj) % L;
-          store_item<D, true>(a.ptr.out[g * L + lp], lo + idx[k], a.n, v[k]);
-        }
-      }
+      for (int k = 0; k < C; ++k)
+        if (val[k]) store_item_rotated<D>(a.ptr.out, g * L, L, l, lo + idx[k], a.n, v[k]);
     }
   }
 }
@@ -701,11 +700,7 @@ __global__ void __launch_bounds__(kThreads) k_hier_wide(const KArgs a) {
 #pragma unroll
       for (int k = 0; k < C; ++k) {
         if (!qval[2 * k]) continue;
-        const uint4 v = quads_to_item<D>(q[2 * k], q[2 * k + 1]);
-        for (int jj = 0; jj < L; ++jj) {
-          const int lp = (l + jj) % L;
-          store_item<D, true>(a.ptr.out[g * L + lp], lo + idx[k], a.n, v);
-        }
+        store_item_rotated<D>(a.ptr.out, g * L, L, l, lo + idx[k], a.n, quads_to_item<D>(q[2 * k], q[2 * k + 1]));
       }
     }
   }
