@@ -796,24 +796,31 @@ def run_reference(args):
             "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# Bytes per rank (KiB) of the selector table's columns: 32 KiB to 8 MiB in
+# powers of two, then 16 and 32 MiB, and 64 MiB for everything above.
+SELECTOR_KIB = (32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536)
+
+
 def run_selector_sweep(args):
     """Every algorithm at every (P, bytes per rank) of the selector table, as
     JSON lines (one per shape). The write-mode kernel is the one this process
-    runs (VRAR_WRITE_KERNEL=plain|staged|async forces one; with staged or
-    async only the write mode is timed)."""
+    runs (VRAR_WRITE_KERNEL=plain|staged|async|batched forces one; with staged,
+    async or batched only the write mode is timed). --sweep-kib limits the
+    sizes."""
     import collective_all_reduce_virtual_b200 as vrar
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     kernel = os.environ.get("VRAR_WRITE_KERNEL", "auto")
+    sizes = [int(k) for k in args.sweep_kib.split(",")] if args.sweep_kib else SELECTOR_KIB
     for P in (2, 4, 8, 16, 32):
-        for kib in (32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384):
+        for kib in sizes:
             spec = dict(DECODE, P=P, n=kib * 512, name=f"P={P} {kib} KiB per rank")
             wl = Workload(spec, device)
             row = {"P": P, "kib": kib, "write_kernel": kernel, "selected": vrar.select_algo(P, wl.n, TDT[wl.dt]),
                    "kernel": vrar.kernel_name(P, wl.n, TDT[wl.dt], "auto")}
-            steps = 200 if kib <= 4096 else 50
-            algos = ("oneshot", "twostage_write", "twostage", "rd") if kernel not in ("staged", "async") \
-                else ("twostage_write",)
+            steps = 200 if kib <= 4096 else 50 if kib <= 16384 else 10
+            algos = ("oneshot", "twostage_write", "twostage", "rd") \
+                if kernel not in ("staged", "async", "batched") else ("twostage_write",)
             for algo in algos:
                 if algo == "rd" and P & (P - 1):
                     continue
@@ -1055,6 +1062,7 @@ def main(argv=None):
                     help="per-call fixed cost and size ladder at 2 and 8 ranks (JSON lines) and exit")
     ap.add_argument("--selector-sweep", action="store_true",
                     help="print per-shape timings of every algorithm (JSON lines) and exit")
+    ap.add_argument("--sweep-kib", metavar="KIB,...", help="bytes per rank (KiB) the selector sweep covers")
     args = ap.parse_args(argv)
     if args.selector_sweep:
         run_selector_sweep(args)

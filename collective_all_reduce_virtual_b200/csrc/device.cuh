@@ -124,6 +124,16 @@ __device__ __forceinline__ uint4 ld_input(const void* p) {
   return v;
 }
 
+// The same load, kept in program order with the other volatile accesses: a
+// batch of these is issued as written, before the arithmetic that uses it.
+__device__ __forceinline__ uint4 ld_input_ordered(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 // Data another CTA of this launch wrote (read after an acquire): L2 only.
 __device__ __forceinline__ uint4 ld_peer(const void* p) {
   uint4 v;

@@ -141,6 +141,94 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
   }
 }
 
+// 2-stage write mode for large messages, with IT items per thread in flight.
+// Same result and work split by rank as k_twostage_write: CTA b of rank r
+// takes passes b, b+B, ... of slice r, a pass being kBatchThreads * IT items
+// (warp w covers items w*32*IT ... of the pass, lane l items l, l+32, ...).
+// For each pass a thread issues the loads of its IT items from eight input
+// ranks at a time before the first add of that batch, so each thread keeps
+// 8 * IT * 16 bytes in flight without shared memory or synchronisation, and
+// the stores of one pass overlap the loads of the next. Rank indices are
+// compile-time (kMaxP is 8, 16 or 32, ranks past P skipped), so the rank
+// pointers are read straight from the kernel parameters. Every full pass runs
+// the unguarded loop; at most one pass per CTA (the one that reaches the end
+// of the slice or the ragged last item) takes the per-item path.
+#ifndef VRAR_BATCH_THREADS
+#define VRAR_BATCH_THREADS 256
+#endif
+#ifndef VRAR_BATCH_MINB
+#define VRAR_BATCH_MINB 2
+#endif
+constexpr int kBatchThreads = VRAR_BATCH_THREADS;
+
+template <class D, int IT, int kMaxP, bool kQ8 = false>
+__global__ void __launch_bounds__(kBatchThreads, VRAR_BATCH_MINB) k_twostage_write_batched(const KArgs a) {
+  constexpr int kSpan = kBatchThreads * IT;
+  pdl_trigger();
+  Cta c = cta_coords(a);
+  const int64_t piece = (a.items + a.P - 1) / a.P;
+  const int64_t lo = lo_of(c.r, piece, a.items), hi = lo_of(c.r + 1, piece, a.items);
+  const int64_t first = lo + static_cast<int64_t>(c.b) * kSpan;
+  if (threadIdx.x < a.P && first < hi)
+    prefetch_items<D>(a.ptr.in[threadIdx.x], first, min(static_cast<int64_t>(kSpan), hi - first), a.n);
+  pdl_wait();
+  if (a.edge_sync) {
+    cta_publish_flag(c, cta_take_ticket(a));
+    if (!block_barrier(a, c, kPhStart)) return;
+  }
+  const int64_t full_hi = min(hi, a.n / D::VE);  // items of the slice wholly inside the vector
+  const int64_t stride = static_cast<int64_t>(a.B) * kSpan;
+  const int64_t lane_off = (threadIdx.x >> 5) * 32 * IT + (threadIdx.x & 31);
+  int64_t base = first;
+  for (; base + kSpan <= full_hi; base += stride) {
+    const int64_t i0 = base + lane_off;  // this thread's items: i0 + 32 t, t < IT
+    Acc<D> acc[IT];
+#pragma unroll
+    for (int q0 = 0; q0 < kMaxP; q0 += 8) {
+      if (q0 < a.P) {
+        uint4 x[IT][8];
+#pragma unroll
+        for (int t = 0; t < IT; ++t) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (q0 + j < a.P) x[t][j] = ld_input_ordered(static_cast<const uint4*>(a.ptr.in[q0 + j]) + i0 + 32 * t);
+        }
+        // Item by item: the last batch's adds of item t, then its stores, so
+        // that only one item's sum is live while the next one's loads land.
+        const bool last = q0 + 8 >= a.P;
+#pragma unroll
+        for (int t = 0; t < IT; ++t) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (q0 + j < a.P) {
+              if (q0 + j == 0) acc[t].template init_in<kQ8>(x[t][j]);
+              else acc[t].template add_in<kQ8>(x[t][j]);
+            }
+          }
+          if (last) {
+            const uint4 v = acc[t].template round_out<kQ8>();
+#pragma unroll
+            for (int q = 0; q < kMaxP; ++q)
+              if (q < a.P) st_stream(static_cast<uint4*>(a.ptr.out[q]) + i0 + 32 * t, v);
+          }
+        }
+      }
+    }
+  }
+  if (base < hi) {  // the one partial pass left to this CTA, if any
+    const int64_t i0 = base + lane_off;
+    for (int t = 0; t < IT; ++t) {
+      const int64_t it = i0 + 32 * t;
+      if (it < hi)
+        store_item_rotated<D>(a.ptr.out, 0, a.P, c.r, it, a.n, reduce_item_out<D, kQ8>(a.ptr, 0, a.P, it, a.n));
+    }
+  }
+  if (a.edge_sync) {
+    __threadfence();
+    block_barrier(a, c, kPhEnd);
+  }
+}
+
 // 2-stage write mode, staged through shared memory with bulk copies. Same
 // result and same work split by rank as k_twostage_write: rank r reduces slice
 // r and streams it to all P outputs. The slice is cut into tiles of

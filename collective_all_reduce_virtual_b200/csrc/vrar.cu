@@ -357,9 +357,9 @@ int launch(KernelFn fn, const KArgs& a, int grid, cudaStream_t stream, int threa
   return VRAR_OK;
 }
 
-// Which write-mode kernel runs: VRAR_WRITE_KERNEL=plain|staged|async forces
-// one (read once); otherwise write_kernel_for() decides by shape.
-enum WriteKernel { kWritePlain = 0, kWriteStaged = 1, kWriteAsync = 2 };
+// Which write-mode kernel runs: VRAR_WRITE_KERNEL=plain|staged|async|batched
+// forces one (read once); otherwise write_kernel_for() decides by shape.
+enum WriteKernel { kWritePlain = 0, kWriteStaged = 1, kWriteAsync = 2, kWriteBatched = 3 };
 
 int write_kernel_override() {
   static int cached = -2;
@@ -369,6 +369,7 @@ int write_kernel_override() {
              : std::strcmp(s, "plain") == 0  ? kWritePlain
              : std::strcmp(s, "staged") == 0 ? kWriteStaged
              : std::strcmp(s, "async") == 0  ? kWriteAsync
+             : std::strcmp(s, "batched") == 0 ? kWriteBatched
                                              : -1;
   }
   return cached;
@@ -377,29 +378,37 @@ int write_kernel_override() {
 // Per-shape choice measured on a B200 (CUDA-graph timings of back-to-back
 // calls, inputs rotated through more than 3x the L2 size): 'O' one-shot,
 // 'A' write mode with the per-thread async-copy kernel, 'S' write mode with
-// the bulk-copy staged kernel, 'P' write mode with the plain kernel. Rows:
-// P <= 2, 4, 8, 16, 32; columns: bytes per rank <= 32 KiB, 64 KiB, ...,
-// 8 MiB, and above. One-shot keeps small messages at two and four ranks (one
-// pass, its re-reads served by L2); at two ranks and 2 MiB per rank the plain
-// write kernel is faster (2.70 against 3.19 us). The async write kernel wins
-// almost everywhere else: every thread keeps all P loads of its items in
-// flight, with no serial issue. From 8 MiB per rank at 4-16 ranks the
-// bulk-copy pipeline streams a little better, and at 32 ranks at 4 and 8 MiB
-// the plain kernel (shared-memory stages of 32 ranks cost occupancy); those
-// margins are a few percent.
-constexpr char kChoice[5][10] = {
-    {'O', 'O', 'O', 'O', 'O', 'O', 'P', 'A', 'A', 'A'},  // P <= 2
-    {'O', 'O', 'A', 'O', 'O', 'A', 'A', 'A', 'S', 'A'},  // P <= 4
-    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 8
-    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S'},  // P <= 16
-    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'A'},  // P <= 32
+// the bulk-copy staged kernel, 'P' write mode with the plain kernel, 'B'
+// write mode with the register-batched kernel. Rows: P <= 2, 4, 8, 16, 32;
+// columns: bytes per rank <= 32 KiB, 64 KiB, ..., 32 MiB, and above. One-shot
+// keeps small messages at two and four ranks (one pass, its re-reads served by
+// L2); at two ranks and 2 MiB per rank the plain write kernel is faster (2.62
+// against 3.19 us). The async write kernel wins almost everywhere else up to a
+// few MiB: every thread keeps all P loads of its items in flight, with no
+// serial issue. From 8 MiB per rank at 4-16 ranks the bulk-copy pipeline
+// streams a little better. Past the L2-sized messages, where every byte comes
+// from DRAM, the plain kernel (one 512-thread CTA per SM, eight loads per
+// thread in flight, stores staggered by rank) streams best at eight ranks and
+// more: 607.6 against 624.0 (batched), 638.3 (async) and 649.2 us (staged) at
+// 8 x 224 MiB, 176.0 against 179.5, 188.0 and 190.0 at 8 x 64 MiB, 180.1
+// against 186.9 (async) at 32 x 16 MiB. At two and four ranks a plain thread
+// has only P loads in flight; there the batched kernel (two items per thread)
+// is fastest above 16 MiB at four ranks (88.1 against 96.2 us at 64 MiB) and
+// above 32 MiB at two.
+constexpr int kChoiceCols = 12;
+constexpr char kChoice[5][kChoiceCols] = {
+    {'O', 'O', 'O', 'O', 'O', 'O', 'P', 'A', 'A', 'A', 'A', 'B'},  // P <= 2
+    {'O', 'O', 'A', 'O', 'O', 'A', 'A', 'A', 'S', 'A', 'B', 'B'},  // P <= 4
+    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S', 'P', 'P'},  // P <= 8
+    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'P', 'P', 'P'},  // P <= 16
+    {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'P', 'P', 'P'},  // P <= 32
 };
 
 char shape_choice(int P, size_t bytes) {
   if (P <= 1) return 'O';
   const int row = P <= 2 ? 0 : P <= 4 ? 1 : P <= 8 ? 2 : P <= 16 ? 3 : 4;
   int col = 0;
-  while (col < 9 && bytes > (static_cast<size_t>(32) << 10 << col)) ++col;
+  while (col < kChoiceCols - 1 && bytes > (static_cast<size_t>(32) << 10 << col)) ++col;
   return kChoice[row][col];
 }
 
@@ -415,7 +424,7 @@ int write_kernel_for(int P, size_t bytes, bool q8 = false) {
   if (forced >= 0) return forced;
   if (q8) return bytes <= (1u << 20) ? kWritePlain : kWriteAsync;
   const char ch = shape_choice(P, bytes);
-  return ch == 'P' ? kWritePlain : ch == 'S' ? kWriteStaged : kWriteAsync;
+  return ch == 'P' ? kWritePlain : ch == 'S' ? kWriteStaged : ch == 'B' ? kWriteBatched : kWriteAsync;
 }
 
 // Async-copy kernel: 64 items (one per thread) per tile, and S tiles in flight
@@ -568,6 +577,24 @@ KernelFn staged_kernel(int ti) {
 KernelFn pick_kernel_dt(vrar_dtype_t dt, vrar_algo_t algo, int C) {
   return dt == VRAR_BF16 ? pick_kernel<Bf16T>(algo, C) : dt == VRAR_FP16 ? pick_kernel<F16T>(algo, C)
                                                                         : pick_kernel<F32T>(algo, C);
+}
+
+// Items each thread of the batched write kernel keeps in flight per input rank.
+#ifndef VRAR_BATCH_ITEMS
+#define VRAR_BATCH_ITEMS 2
+#endif
+
+template <class D, bool Q>
+KernelFn batched_kernel(int P) {
+  return P <= 8    ? k_twostage_write_batched<D, VRAR_BATCH_ITEMS, 8, Q>
+         : P <= 16 ? k_twostage_write_batched<D, VRAR_BATCH_ITEMS, 16, Q>
+                   : k_twostage_write_batched<D, VRAR_BATCH_ITEMS, 32, Q>;
+}
+
+KernelFn batched_kernel_dt(vrar_dtype_t dt, int P, bool q8) {
+  if (dt == VRAR_BF16) return q8 ? batched_kernel<Bf16T, true>(P) : batched_kernel<Bf16T, false>(P);
+  if (dt == VRAR_FP16) return q8 ? batched_kernel<F16T, true>(P) : batched_kernel<F16T, false>(P);
+  return batched_kernel<F32T, false>(P);
 }
 
 KernelFn staged_kernel_dt(vrar_dtype_t dt, int ti, bool q8) {
@@ -850,6 +877,15 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     a.B = B;
     return launch(sf, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), 32 + ti, smem);
   }
+  if (wk == kWriteBatched) {
+    KernelFn bf = batched_kernel_dt(dtype, P, q8);
+    const int64_t passes = std::max<int64_t>(1, (work + kBatchThreads * VRAR_BATCH_ITEMS - 1) /
+                                                    (kBatchThreads * VRAR_BATCH_ITEMS));
+    const int resident = grid_budget(bf, dev, sms, kBatchThreads);
+    if (resident < 1) return VRAR_ECUDA;
+    a.B = static_cast<int>(std::min<int64_t>(passes, std::max(1, std::min(resident, kMaxCtas) / P)));
+    return launch(bf, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), kBatchThreads);
+  }
   int threads = kThreads;
   if (algo == VRAR_ALGO_ONESHOT && static_cast<size_t>(P) * n * elem_size(dtype) <= kOneshotSmallBytes)
     threads = kSmallThreads;
@@ -957,8 +993,10 @@ const char* vrar_kernel_name(int P, size_t n, vrar_dtype_t dtype, vrar_algo_t al
     case VRAR_ALGO_TWOSTAGE: return "k_twostage";
     case VRAR_ALGO_TWOSTAGE_WRITE: {
       const int wk = write_kernel_for(P, n * elem_size(dtype), g_set.fp8_quant.load() != 0 && dtype != VRAR_FP32);
-      return wk == kWriteAsync ? "k_twostage_write_async" : wk == kWriteStaged ? "k_twostage_write_staged"
-                                                                                : "k_twostage_write";
+      return wk == kWriteAsync     ? "k_twostage_write_async"
+             : wk == kWriteStaged  ? "k_twostage_write_staged"
+             : wk == kWriteBatched ? "k_twostage_write_batched"
+                                   : "k_twostage_write";
     }
     case VRAR_ALGO_RD: return wide_wire(algo, dtype) ? "k_rd_wide" : "k_rd";
     case VRAR_ALGO_HIER: return wide_wire(algo, dtype) ? "k_hier_wide" : "k_hier";

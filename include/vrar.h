@@ -154,10 +154,11 @@ VRAR_API int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype);
  * Base name of the kernel that vrar_allreduce(.., P, n, dtype, algo, ..) would
  * launch under the current settings (AUTO resolved as vrar_allreduce resolves
  * it, the payload wire, the VRAR_WRITE_KERNEL override), e.g.
- * "k_twostage_write_async". Write mode has three kernels with one result:
- * "k_twostage_write" (plain), "k_twostage_write_staged" (bulk copies into
- * shared memory by one producer lane), "k_twostage_write_async" (per-thread
- * async copies into shared memory), chosen per shape from the same measured
+ * "k_twostage_write_async". Write mode has four kernels with one result:
+ * "k_twostage_write" (plain: one item per thread and pass), "k_twostage_write_staged"
+ * (bulk copies into shared memory by one producer lane), "k_twostage_write_async"
+ * (per-thread async copies into shared memory), "k_twostage_write_batched" (two
+ * items per thread and pass), chosen per shape from the same measured
  * table as vrar_select_algo (with fp8 payloads on: the plain kernel up to 1 MiB per
  * rank, the async kernel above). For profilers and benchmarks; the sources have
  * no counterpart. Returns a static string, or NULL for invalid arguments

@@ -150,7 +150,9 @@ def test_selector_table_entries():
     assert vrar.select_algo(2, 1 << 19, bf) == "oneshot"            # 1 MiB at 2 ranks
     assert vrar.select_algo(2, 1 << 20, bf) == "twostage_write"     # 2 MiB at 2 ranks (plain write kernel)
     assert vrar.kernel_name(2, 1 << 20, bf, "auto") == "k_twostage_write"
-    assert vrar.kernel_name(32, 8 << 20, bf, "auto") == "k_twostage_write_async"  # 16 MiB at 32 ranks
+    assert vrar.kernel_name(32, 8 << 20, bf, "auto") == "k_twostage_write"        # 16 MiB at 32 ranks
+    assert vrar.kernel_name(4, 32 << 20, bf, "auto") == "k_twostage_write_batched"  # 64 MiB at 4 ranks
+    assert vrar.kernel_name(2, 16 << 20, bf, "auto") == "k_twostage_write_async"    # 32 MiB at 2 ranks
     assert vrar.select_algo(2, 4 << 20, bf) == "twostage_write"     # 8 MiB at 2 ranks
     assert vrar.select_algo(8, 524288, bf) == "twostage_write"      # 1 MiB at 8 ranks (the decode shape)
     assert vrar.select_algo(8, 117440512, bf) == "twostage_write"   # prefill
@@ -159,7 +161,7 @@ def test_selector_table_entries():
 
 
 def test_kernel_name():
-    """Which kernel a call launches: write mode has three kernels with one result."""
+    """Which kernel a call launches: write mode has four kernels with one result."""
     bf = torch.bfloat16
     if os.environ.get("VRAR_WRITE_KERNEL") or os.environ.get("VRAR_ALGO"):
         pytest.skip("an override is set in the environment")
@@ -168,7 +170,8 @@ def test_kernel_name():
     assert vrar.kernel_name(8, 524288, bf, "rd") == "k_rd"
     assert vrar.kernel_name(32, 524288, bf, "hier") == "k_hier"
     assert vrar.kernel_name(8, 524288, bf, "auto") == "k_twostage_write_async"       # the decode shape
-    assert vrar.kernel_name(8, 117440512, bf, "auto") == "k_twostage_write_staged"   # prefill
+    assert vrar.kernel_name(8, 117440512, bf, "auto") == "k_twostage_write"          # prefill
+    assert vrar.kernel_name(8, 8 << 20, bf, "auto") == "k_twostage_write_staged"     # 16 MiB at 8 ranks
     assert vrar.kernel_name(1, 1000, bf, "auto") == "k_oneshot"
     for P in (1, 2, 3, 8, 13, 32):
         for n in (0, 1, 65536, 524288, 1 << 24):

@@ -179,7 +179,7 @@ CHILD = textwrap.dedent("""
 """)
 
 
-@pytest.mark.parametrize("variant", ["plain", "staged", "async"])
+@pytest.mark.parametrize("variant", ["plain", "staged", "async", "batched"])
 def test_fp8_each_write_kernel(variant):
     env = dict(os.environ, VRAR_WRITE_KERNEL=variant)
     code = CHILD.format(root=ROOT, tests=os.path.join(ROOT, "tests"))

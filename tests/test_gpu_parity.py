@@ -419,6 +419,8 @@ def test_spin_stats_count_timeouts():
     ("twostage", 4, 8, False, 2, 40_000),
     ("twostage_write", 8, 8, True, 1, 40_000),      # async-copy write kernel
     ("twostage_write", 8, 8, True, 1, 4_194_304),   # 8 MiB per rank: bulk-copy staged kernel
+    ("twostage_write", 8, 8, True, 1, 20_000_000),  # 40 MiB per rank: plain kernel
+    ("twostage_write", 4, 8, True, 1, 20_000_000),  # 40 MiB per rank at 4 ranks: batched kernel
     ("rd", 4, 8, True, 4, 40_000),
     ("hier", 8, 2, True, 4, 40_000),
     ("hier", 8, 2, True, 4, 600_000),               # above 256 KiB per rank: two CTAs per SM
@@ -428,7 +430,8 @@ def test_missing_rank_times_out_and_recovers(algo, P, L, edge, phase, n):
     kernel records VRAR_ETIMEDOUT and exits, and the next call works."""
     xs = gen(P, n, "bf16", synth.normal(0.0, 1.0), seed=5)
     if algo == "twostage_write":  # the case must reach the kernel it is there for
-        want_kernel = {40_000: "k_twostage_write_async", 4_194_304: "k_twostage_write_staged"}[n]
+        want_kernel = {(8, 40_000): "k_twostage_write_async", (8, 4_194_304): "k_twostage_write_staged",
+                       (8, 20_000_000): "k_twostage_write", (4, 20_000_000): "k_twostage_write_batched"}[(P, n)]
         assert vrar.kernel_name(P, n, torch.bfloat16, algo) == want_kernel
     d_in = _dev(xs, "bf16")
     vrar.set_group_size(L)

@@ -8,10 +8,10 @@ exactly the full-size results at those indices. Rank 0's output is compared
 with the oracle element by element over all 117,440,512 elements; the other
 P - 1 outputs are compared with rank 0's, whole, on the device.
 
-The write mode has three kernels; the per-shape table gives this shape to the
-bulk-copy staged kernel. The async-copy and plain kernels are forced in child
-processes (VRAR_WRITE_KERNEL is read once per process), so that every write
-kernel is checked at this size.
+The write mode has four kernels; the per-shape table gives this shape to the
+plain kernel. The staged, async-copy and register-batched kernels are forced
+in child processes (VRAR_WRITE_KERNEL is read once per process), so that every
+write kernel is checked at this size.
 """
 
 import os
@@ -73,12 +73,12 @@ def _run(cases, env_extra=None):
     assert res.returncode == 0 and "ok" in res.stdout, res.stdout[-2000:] + res.stderr[-4000:]
 
 
-def test_prefill_full_pull_and_staged_write():
-    """The pull 2-stage and the write mode as the table picks it (staged kernel)."""
-    _run([("twostage", "k_twostage"), ("twostage_write", "k_twostage_write_staged"),
-          ("auto", "k_twostage_write_staged")])
+def test_prefill_full_pull_and_plain_write():
+    """The pull 2-stage and the write mode as the table picks it (plain kernel)."""
+    _run([("twostage", "k_twostage"), ("twostage_write", "k_twostage_write"), ("auto", "k_twostage_write")])
 
 
-@pytest.mark.parametrize("variant,kernel", [("async", "k_twostage_write_async"), ("plain", "k_twostage_write")])
+@pytest.mark.parametrize("variant,kernel", [("staged", "k_twostage_write_staged"), ("async", "k_twostage_write_async"),
+                                            ("batched", "k_twostage_write_batched")])
 def test_prefill_full_other_write_kernels(variant, kernel):
     _run([("twostage_write", kernel)], {"VRAR_WRITE_KERNEL": variant})

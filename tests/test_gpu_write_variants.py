@@ -1,11 +1,13 @@
-"""The three write-mode kernels (plain, bulk-copy staged, per-thread async
-copies) against the oracle.
+"""The four write-mode kernels (plain, bulk-copy staged, per-thread async
+copies, register-batched) against the oracle.
 
 The per-shape table sends each shape to one of the kernels, so this test
 forces each in turn (VRAR_WRITE_KERNEL is read once per process, hence the
 child processes) over shapes with ragged tails, up to 32 ranks, all three
 dtypes, with and without the start/end barriers, and with a CTA budget (which
 changes the grid and, for the staged and async kernels, the stage depth).
+The batched kernel's unguarded passes need 512 items per CTA pass, so the
+larger shapes at 13, 16, 24 and 32 ranks run both its paths.
 """
 
 import os
@@ -28,8 +30,8 @@ CHILD = textwrap.dedent("""
     import oracle, synth
     from util import from_np, gen, to_np, bits_of
     for dtype in ("bf16", "fp32", "fp16"):
-        for P, n in ((1, 1001), (2, 7), (3, 66_001), (8, 9), (8, 300_007), (13, 4_099), (16, 70_001), (24, 50_021),
-                     (32, 33_333), (32, 1_000_003)):
+        for P, n in ((1, 1001), (2, 7), (3, 66_001), (8, 9), (8, 300_007), (13, 4_099), (13, 700_001), (16, 70_001),
+                     (24, 50_021), (24, 2_000_003), (32, 33_333), (32, 1_000_003)):
             xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P + n)
             want = oracle.allreduce("twostage_write", xs, dtype)
             for edge, cap in ((False, 0), (True, 0), (False, 64)):
@@ -46,7 +48,7 @@ CHILD = textwrap.dedent("""
 """)
 
 
-@pytest.mark.parametrize("variant", ["plain", "staged", "async"])
+@pytest.mark.parametrize("variant", ["plain", "staged", "async", "batched"])
 def test_write_kernel_variant_matches_oracle(variant):
     env = dict(os.environ, VRAR_WRITE_KERNEL=variant)
     code = CHILD.format(root=ROOT, tests=os.path.join(ROOT, "tests"))
