@@ -114,8 +114,8 @@ __global__ void __launch_bounds__(T) k_twostage(const KArgs a) {
 // and change 3]: rank r reduces slice r and streams the result straight into
 // all P outputs; a device-scope fence then makes those stores visible before
 // the end barrier's flags. kQ8: inputs and reduced slice pass the fp8 wire.
-template <class D, bool kQ8 = false>
-__global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
+template <class D, bool kQ8>
+__device__ __forceinline__ void twostage_write_plain(const KArgs& a) {
   pdl_trigger();
   Cta c = cta_coords(a);
   {
@@ -141,6 +141,21 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
   }
 }
 
+// The plain write kernel, registers left to the compiler (78 for bf16): one
+// 512-thread CTA per SM, the build that streams DRAM-sized calls best.
+template <class D, bool kQ8 = false>
+__global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
+  twostage_write_plain<D, kQ8>(a);
+}
+
+// The same kernel with its registers budgeted for kMinBlocks CTAs per SM, for
+// small calls that one CTA per SM cannot cover in one pass (same name: an
+// overload of the template above by its parameter list).
+template <class D, bool kQ8, int kMinBlocks>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) k_twostage_write(const KArgs a) {
+  twostage_write_plain<D, kQ8>(a);
+}
+
 // 2-stage write mode for large messages, with IT items per thread in flight.
 // Same result and work split by rank as k_twostage_write: CTA b of rank r
 // takes passes b, b+B, ... of slice r, a pass being kBatchThreads * IT items
@@ -153,6 +168,8 @@ __global__ void __launch_bounds__(kThreads) k_twostage_write(const KArgs a) {
 // pointers are read straight from the kernel parameters. Every full pass runs
 // the unguarded loop; at most one pass per CTA (the one that reaches the end
 // of the slice or the ragged last item) takes the per-item path.
+// Threads per CTA and the CTAs per SM its register budget is sized for
+// (compile-time; the defaults, two 256-thread CTAs per SM, measured fastest).
 #ifndef VRAR_BATCH_THREADS
 #define VRAR_BATCH_THREADS 256
 #endif

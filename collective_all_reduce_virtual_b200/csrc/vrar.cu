@@ -382,8 +382,8 @@ int write_kernel_override() {
 // write mode with the register-batched kernel. Rows: P <= 2, 4, 8, 16, 32;
 // columns: bytes per rank <= 32 KiB, 64 KiB, ..., 32 MiB, and above. One-shot
 // keeps small messages at two and four ranks (one pass, its re-reads served by
-// L2); at two ranks and 2 MiB per rank the plain write kernel is faster (2.62
-// against 3.19 us). The async write kernel wins almost everywhere else up to a
+// L2); at two ranks and 2 MiB per rank the plain write kernel is faster (2.35
+// against 3.19 us, in its two-CTA-per-SM build). The async write kernel wins almost everywhere else up to a
 // few MiB: every thread keeps all P loads of its items in flight, with no
 // serial issue. From 8 MiB per rank at 4-16 ranks the bulk-copy pipeline
 // streams a little better. Past the L2-sized messages, where every byte comes
@@ -459,11 +459,22 @@ constexpr int kSmallThreads = 128;
 // mid barrier (measured 6-10 % faster than 512 from 128 KiB to 2 MiB per rank).
 constexpr int kPullThreads = 256;
 
+// The plain write kernel budgets its registers for one 512-thread CTA per SM,
+// which streams DRAM-sized calls best (608 against 638 us with two at
+// 8 x 224 MiB, 180 against 199 us at 32 x 16 MiB, 48.3 against 49.5 us at
+// 32 x 4 MiB). A call that moves at most this many bytes (2 P n s) and that one
+// CTA per SM cannot cover in one pass takes the two-CTA build instead (at 2 ranks
+// x 2 MiB: 256 CTAs in one pass, 2.36 against 3.60 us; x 4 MiB: 4.62 against
+// 6.39 us); one that fits in one pass keeps one CTA per SM (2 x 1 MiB: 2.03
+// against 2.51 us).
+constexpr size_t kPlainTwoPerSmBytes = 32u << 20;
+
 // Kernels of the custom all-reduce (one-shot, pull 2-stage, plain write), with
 // or without the fp8 wire (q8, 16-bit element types only; the host rejects
-// fp8 for fp32 before it gets here).
+// fp8 for fp32 before it gets here). two_per_sm picks the plain write kernel's
+// two-CTA budget (not with q8).
 template <class D>
-KernelFn custom_kernel(vrar_algo_t algo, int threads, bool q8) {
+KernelFn custom_kernel(vrar_algo_t algo, int threads, bool q8, bool two_per_sm = false) {
   if constexpr (D::VE == 8) {
     if (q8) {
       if (algo == VRAR_ALGO_ONESHOT)
@@ -474,13 +485,13 @@ KernelFn custom_kernel(vrar_algo_t algo, int threads, bool q8) {
   }
   if (algo == VRAR_ALGO_ONESHOT) return threads == kSmallThreads ? k_oneshot<D, kSmallThreads> : k_oneshot<D>;
   if (algo == VRAR_ALGO_TWOSTAGE) return k_twostage<D, kPullThreads>;
-  return k_twostage_write<D>;
+  return two_per_sm ? k_twostage_write<D, false, 2> : k_twostage_write<D>;
 }
 
-KernelFn custom_kernel_dt(vrar_dtype_t dt, vrar_algo_t algo, int threads, bool q8) {
-  return dt == VRAR_BF16   ? custom_kernel<Bf16T>(algo, threads, q8)
-         : dt == VRAR_FP16 ? custom_kernel<F16T>(algo, threads, q8)
-                           : custom_kernel<F32T>(algo, threads, false);
+KernelFn custom_kernel_dt(vrar_dtype_t dt, vrar_algo_t algo, int threads, bool q8, bool two_per_sm = false) {
+  return dt == VRAR_BF16   ? custom_kernel<Bf16T>(algo, threads, q8, two_per_sm)
+         : dt == VRAR_FP16 ? custom_kernel<F16T>(algo, threads, q8, two_per_sm)
+                           : custom_kernel<F32T>(algo, threads, false, two_per_sm);
 }
 
 // HIER (element wire) by size, measured at 4 groups x 8 ranks: up to 256 KiB
@@ -891,7 +902,13 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
     threads = kSmallThreads;
   if (algo == VRAR_ALGO_TWOSTAGE) threads = kPullThreads;
   fn = custom_kernel_dt(dtype, algo, threads, q8);
-  a.B = blocks_per_rank(work, P, grid_budget(fn, dev, sms, threads), threads);
+  int budget = grid_budget(fn, dev, sms, threads);
+  if (algo == VRAR_ALGO_TWOSTAGE_WRITE && !q8 && 2 * static_cast<size_t>(P) * n * elem_size(dtype) <= kPlainTwoPerSmBytes &&
+      work > static_cast<int64_t>(std::min(budget, kMaxCtas) / P) * threads) {
+    fn = custom_kernel_dt(dtype, algo, threads, false, true);  // one pass needs two CTAs per SM
+    budget = grid_budget(fn, dev, sms, threads);
+  }
+  a.B = blocks_per_rank(work, P, budget, threads);
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), threads);
 }
 

@@ -7,7 +7,9 @@ child processes) over shapes with ragged tails, up to 32 ranks, all three
 dtypes, with and without the start/end barriers, and with a CTA budget (which
 changes the grid and, for the staged and async kernels, the stage depth).
 The batched kernel's unguarded passes need 512 items per CTA pass, so the
-larger shapes at 13, 16, 24 and 32 ranks run both its paths.
+larger shapes at 13, 16, 24 and 32 ranks run both its paths; 2 ranks x 2 MiB
+is a small call that one plain CTA per SM cannot cover in one pass, so the
+plain kernel runs its two-CTA-per-SM build there.
 """
 
 import os
@@ -30,8 +32,8 @@ CHILD = textwrap.dedent("""
     import oracle, synth
     from util import from_np, gen, to_np, bits_of
     for dtype in ("bf16", "fp32", "fp16"):
-        for P, n in ((1, 1001), (2, 7), (3, 66_001), (8, 9), (8, 300_007), (13, 4_099), (13, 700_001), (16, 70_001),
-                     (24, 50_021), (24, 2_000_003), (32, 33_333), (32, 1_000_003)):
+        for P, n in ((1, 1001), (2, 7), (2, 1_048_583), (3, 66_001), (8, 9), (8, 300_007), (13, 4_099), (13, 700_001),
+                     (16, 70_001), (24, 50_021), (24, 2_000_003), (32, 33_333), (32, 1_000_003)):
             xs = gen(P, n, dtype, synth.normal(0.0, 1.0), seed=P + n)
             want = oracle.allreduce("twostage_write", xs, dtype)
             for edge, cap in ((False, 0), (True, 0), (False, 64)):
