@@ -382,10 +382,11 @@ int write_kernel_override() {
 // write mode with the register-batched kernel. Rows: P <= 2, 4, 8, 16, 32;
 // columns: bytes per rank <= 32 KiB, 64 KiB, ..., 32 MiB, and above. One-shot
 // keeps small messages at two and four ranks (one pass, its re-reads served by
-// L2); at two ranks and 2 MiB per rank the plain write kernel is faster (2.35
-// against 3.19 us, in its two-CTA-per-SM build). The async write kernel wins almost everywhere else up to a
-// few MiB: every thread keeps all P loads of its items in flight, with no
-// serial issue. From 8 MiB per rank at 4-16 ranks the bulk-copy pipeline
+// L2); at two and four ranks and 2 MiB per rank the batched write kernel is
+// faster (2.27 against one-shot's 3.19 us at two ranks, 3.23 against the
+// async kernel's 3.46 at four). The async write kernel wins almost everywhere
+// else up to a few MiB: every thread keeps all P loads of its items in flight,
+// with no serial issue. From 8 MiB per rank at 4-16 ranks the bulk-copy pipeline
 // streams a little better. Past the L2-sized messages, where every byte comes
 // from DRAM, the plain kernel (one 512-thread CTA per SM, eight loads per
 // thread in flight, stores staggered by rank) streams best at eight ranks and
@@ -397,8 +398,8 @@ int write_kernel_override() {
 // above 32 MiB at two.
 constexpr int kChoiceCols = 12;
 constexpr char kChoice[5][kChoiceCols] = {
-    {'O', 'O', 'O', 'O', 'O', 'O', 'P', 'A', 'A', 'A', 'A', 'B'},  // P <= 2
-    {'O', 'O', 'A', 'O', 'O', 'A', 'A', 'A', 'S', 'A', 'B', 'B'},  // P <= 4
+    {'O', 'O', 'O', 'O', 'O', 'O', 'B', 'A', 'A', 'A', 'A', 'B'},  // P <= 2
+    {'O', 'O', 'A', 'O', 'O', 'A', 'B', 'A', 'S', 'A', 'B', 'B'},  // P <= 4
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'S', 'P', 'P'},  // P <= 8
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'A', 'S', 'P', 'P', 'P'},  // P <= 16
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'P', 'P', 'P'},  // P <= 32

@@ -148,8 +148,8 @@ def test_selector_table_entries():
     bf = torch.bfloat16
     assert vrar.select_algo(1, 1 << 20, bf) == "oneshot"            # a copy
     assert vrar.select_algo(2, 1 << 19, bf) == "oneshot"            # 1 MiB at 2 ranks
-    assert vrar.select_algo(2, 1 << 20, bf) == "twostage_write"     # 2 MiB at 2 ranks (plain write kernel)
-    assert vrar.kernel_name(2, 1 << 20, bf, "auto") == "k_twostage_write"
+    assert vrar.select_algo(2, 1 << 20, bf) == "twostage_write"     # 2 MiB at 2 ranks (batched write kernel)
+    assert vrar.kernel_name(2, 1 << 20, bf, "auto") == "k_twostage_write_batched"  # 2 MiB at 2 ranks
     assert vrar.kernel_name(32, 8 << 20, bf, "auto") == "k_twostage_write"        # 16 MiB at 32 ranks
     assert vrar.kernel_name(4, 32 << 20, bf, "auto") == "k_twostage_write_batched"  # 64 MiB at 4 ranks
     assert vrar.kernel_name(2, 16 << 20, bf, "auto") == "k_twostage_write_async"    # 32 MiB at 2 ranks
