@@ -806,23 +806,26 @@ def run_selector_sweep(args):
     JSON lines (one per shape). The write-mode kernel is the one this process
     runs (VRAR_WRITE_KERNEL=plain|staged|async|batched forces one; with staged,
     async or batched only the write mode is timed). --sweep-kib limits the
-    sizes."""
+    sizes; --fp8 turns the fp8 payloads on (one-shot, write mode and the pull
+    2-stage; recursive doubling has no fp8 form)."""
     import collective_all_reduce_virtual_b200 as vrar
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     kernel = os.environ.get("VRAR_WRITE_KERNEL", "auto")
     sizes = [int(k) for k in args.sweep_kib.split(",")] if args.sweep_kib else SELECTOR_KIB
+    vrar.set_fp8_quant(bool(args.fp8))
     for P in (2, 4, 8, 16, 32):
         for kib in sizes:
             spec = dict(DECODE, P=P, n=kib * 512, name=f"P={P} {kib} KiB per rank")
             wl = Workload(spec, device)
-            row = {"P": P, "kib": kib, "write_kernel": kernel, "selected": vrar.select_algo(P, wl.n, TDT[wl.dt]),
+            row = {"P": P, "kib": kib, "write_kernel": kernel, "fp8": bool(args.fp8),
+                   "selected": vrar.select_algo(P, wl.n, TDT[wl.dt]),
                    "kernel": vrar.kernel_name(P, wl.n, TDT[wl.dt], "auto")}
             steps = 200 if kib <= 4096 else 50 if kib <= 16384 else 10
             algos = ("oneshot", "twostage_write", "twostage", "rd") \
                 if kernel not in ("staged", "async", "batched") else ("twostage_write",)
             for algo in algos:
-                if algo == "rd" and P & (P - 1):
+                if algo == "rd" and (P & (P - 1) or args.fp8):
                     continue
                 row[algo] = round(min(measure_algo(wl, algo, steps, 3) for _ in range(3)) * 1e3, 3)
             wl.free()
@@ -1063,6 +1066,7 @@ def main(argv=None):
     ap.add_argument("--selector-sweep", action="store_true",
                     help="print per-shape timings of every algorithm (JSON lines) and exit")
     ap.add_argument("--sweep-kib", metavar="KIB,...", help="bytes per rank (KiB) the selector sweep covers")
+    ap.add_argument("--fp8", action="store_true", help="selector sweep with fp8 payloads on")
     args = ap.parse_args(argv)
     if args.selector_sweep:
         run_selector_sweep(args)

@@ -405,26 +405,43 @@ constexpr char kChoice[5][kChoiceCols] = {
     {'A', 'A', 'A', 'A', 'A', 'A', 'A', 'P', 'P', 'P', 'P', 'P'},  // P <= 32
 };
 
-char shape_choice(int P, size_t bytes) {
-  if (P <= 1) return 'O';
+// The write-mode kernel with fp8 payloads on, measured the same way (rows and
+// columns as kChoice). With fp8 the kernels are bound by the quantisation
+// arithmetic (P + 1 groups of 8 per item), not by memory, so what counts is
+// the warps each SM keeps issuing. The async kernel wins small messages. Its
+// shared-memory stages grow with P and cut its CTAs per SM, so from 512 KiB -
+// 1 MiB per rank at 16 and 32 ranks the plain kernel's 512-thread CTAs win
+// (at 32 ranks x 2 MiB: 62.2 against 133.1 us async; x 64 MiB: 1927 against 3711);
+// at 4 ranks from 1 MiB the staged kernel (226 against 240 us async at
+// 64 MiB); at 8 ranks the async kernel from 4 MiB (410 against 445 us plain at
+// 64 MiB).
+constexpr char kChoiceFp8[5][kChoiceCols] = {
+    {'A', 'A', 'A', 'A', 'P', 'P', 'A', 'A', 'A', 'A', 'A', 'A'},  // P <= 2
+    {'A', 'A', 'A', 'A', 'A', 'S', 'S', 'S', 'S', 'S', 'S', 'S'},  // P <= 4
+    {'A', 'A', 'A', 'A', 'A', 'P', 'B', 'A', 'A', 'A', 'A', 'A'},  // P <= 8
+    {'A', 'A', 'A', 'A', 'A', 'P', 'P', 'P', 'P', 'P', 'P', 'P'},  // P <= 16
+    {'A', 'A', 'A', 'A', 'P', 'P', 'P', 'P', 'P', 'P', 'P', 'P'},  // P <= 32
+};
+
+char table_choice(const char (&table)[5][kChoiceCols], int P, size_t bytes) {
   const int row = P <= 2 ? 0 : P <= 4 ? 1 : P <= 8 ? 2 : P <= 16 ? 3 : 4;
   int col = 0;
   while (col < kChoiceCols - 1 && bytes > (static_cast<size_t>(32) << 10 << col)) ++col;
-  return kChoice[row][col];
+  return table[row][col];
 }
+
+char shape_choice(int P, size_t bytes) { return P <= 1 ? 'O' : table_choice(kChoice, P, bytes); }
 
 // Which write-mode kernel runs a TWOSTAGE_WRITE call. Shapes the table gives
 // to one-shot (when write mode is asked for by name) take the async kernel,
 // the fastest write kernel on small messages. With fp8 payloads (q8) the
-// kernels are bound by the quantisation arithmetic, not by memory: the plain
-// kernel's 512-thread CTAs keep the most arithmetic in flight up to 1 MiB per
-// rank, the async kernel above (measured at 8 ranks: 9.5 against 12.2 us at
-// 1 MiB; 18.1, 56 and 185 us against 18.3, 71 and 214 at 2, 8 and 28 MiB).
+// kernel comes from kChoiceFp8; the algorithm AUTO runs does not depend on
+// fp8 (one-shot and write mode pass different values through the fp8 wire, so
+// the result stays a function of the shape alone).
 int write_kernel_for(int P, size_t bytes, bool q8 = false) {
   const int forced = write_kernel_override();
   if (forced >= 0) return forced;
-  if (q8) return bytes <= (1u << 20) ? kWritePlain : kWriteAsync;
-  const char ch = shape_choice(P, bytes);
+  const char ch = q8 ? table_choice(kChoiceFp8, P, bytes) : shape_choice(P, bytes);
   return ch == 'P' ? kWritePlain : ch == 'S' ? kWriteStaged : ch == 'B' ? kWriteBatched : kWriteAsync;
 }
 

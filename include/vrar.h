@@ -159,8 +159,8 @@ VRAR_API int vrar_select_algo(int P, size_t n, vrar_dtype_t dtype);
  * (bulk copies into shared memory by one producer lane), "k_twostage_write_async"
  * (per-thread async copies into shared memory), "k_twostage_write_batched" (two
  * items per thread and pass), chosen per shape from the same measured
- * table as vrar_select_algo (with fp8 payloads on: the plain kernel up to 1 MiB per
- * rank, the async kernel above). For profilers and benchmarks; the sources have
+ * table as vrar_select_algo (with fp8 payloads on, from a second measured table:
+ * the algorithm AUTO runs stays the same). For profilers and benchmarks; the sources have
  * no counterpart. Returns a static string, or NULL for invalid arguments
  * (P outside 1..VRAR_MAX_RANKS, unknown dtype or algorithm). Launches nothing.
  */

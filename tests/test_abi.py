@@ -188,6 +188,29 @@ def test_kernel_name():
             vrar.kernel_name(bad[0], bad[1], bf, "auto")
 
 
+def test_fp8_write_kernel_table():
+    """With fp8 payloads on, the write kernel comes from its own measured table
+    (the arithmetic, not memory, bounds it); the algorithm AUTO runs does not
+    change (one-shot and write mode pass different values through the wire)."""
+    bf = torch.bfloat16
+    if os.environ.get("VRAR_WRITE_KERNEL") or os.environ.get("VRAR_ALGO"):
+        pytest.skip("an override is set in the environment")
+    algos = {(P, n): vrar.select_algo(P, n, bf) for P in (2, 4, 8, 32) for n in (1 << 14, 1 << 20, 1 << 24)}
+    vrar.set_fp8_quant(True)
+    try:
+        assert vrar.kernel_name(32, 1 << 20, bf, "twostage_write") == "k_twostage_write"          # 32 x 2 MiB
+        assert vrar.kernel_name(32, 1 << 16, bf, "twostage_write") == "k_twostage_write_async"    # 32 x 128 KiB
+        assert vrar.kernel_name(8, 1 << 19, bf, "twostage_write") == "k_twostage_write"           # 8 x 1 MiB
+        assert vrar.kernel_name(8, 1 << 20, bf, "twostage_write") == "k_twostage_write_batched"   # 8 x 2 MiB
+        assert vrar.kernel_name(8, 1 << 21, bf, "twostage_write") == "k_twostage_write_async"     # 8 x 4 MiB
+        assert vrar.kernel_name(4, 1 << 23, bf, "twostage_write") == "k_twostage_write_staged"    # 4 x 16 MiB
+        assert vrar.kernel_name(8, 117440512, bf, "auto") == "k_twostage_write_async"             # prefill
+        assert {(P, n): vrar.select_algo(P, n, bf) for P, n in algos} == algos
+    finally:
+        vrar.set_fp8_quant(False)
+    assert vrar.kernel_name(8, 117440512, bf, "auto") == "k_twostage_write"
+
+
 def test_payload_wire_setting():
     assert vrar.get_payload_wire() == "element"
     assert L.vrar_set_payload_wire(7) == vrar.EINVAL
