@@ -321,11 +321,37 @@ __device__ __forceinline__ void e4m3_round2(float& lo, float& hi) {
   hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
 }
 
+// The group scale amax / 448, rounded to nearest even, for 2^-120 <= amax <=
+// FLT_MAX: the product by c = RN(1/448) = 0x1.24924ap-9, corrected once by its
+// exact remainder (Markstein's FMA correction step: r = x - q0 * 448 is exact
+// in one fma, and q0 + r * c rounds to the quotient). Checked against the
+// exactly rounded quotient for every binary32 in that range (the test suite
+// runs the same formula over all of them); below 2^-120 the quotient is deep in
+// the subnormal range, where the correction can be off by one unit, and the
+// caller divides instead.
+__device__ __forceinline__ float div448_rn(float x) {
+  const float c = 0x1.24924ap-9f;
+  const float q0 = __fmul_rn(x, c);
+  const float r = __fmaf_rn(-q0, 448.0f, x);
+  return __fmaf_rn(r, c, q0);
+}
+
+// 1/s to within 2^-23 relative, for s and 1/s normal: the hardware's
+// approximate reciprocal and one Newton-Raphson step (e = 1 - s r0 in one fma,
+// r1 = r0 + r0 e), whose error is the square of the approximation's plus one
+// rounding.
+__device__ __forceinline__ float recip_nr(float s) {
+  float r0;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r0) : "f"(s));
+  const float e = __fmaf_rn(-s, r0, 1.0f);
+  return __fmaf_rn(r0, e, r0);
+}
+
 // E4M3(x / s) needs the binary32 quotient x / s only up to which side of an
-// E4M3 rounding midpoint it falls. The product t = x * r with r = 1/s (both
-// rounded to nearest) is within 3 units in the last place of the quotient
-// (two roundings of 2^-24 relative each, for r a normal number), so it rounds
-// to the same E4M3 value unless a midpoint lies within 3 units of it. Where t
+// E4M3 rounding midpoint it falls. The product t = x * r with r within 2^-23
+// of 1/s (relative) is within 3 units in the last place of the quotient (that
+// error and one rounding of 2^-24), so it rounds to the same E4M3 value
+// unless a midpoint lies within 3 units of it. Where t
 // is within 8 units of a midpoint of a normal E4M3 binade (its 20 fraction bits
 // below the 3 that E4M3 keeps are within 8 of 1000...0), or in E4M3's
 // subnormal range (below 2^-6, where the midpoints sit elsewhere), the exact
@@ -342,17 +368,17 @@ __device__ __forceinline__ float fp8_quotient(float x, float s, float r) {
 // The fp8 wire on one group of 8 binary32 values, in place: s = amax / 448
 // (1 when that is 0), each value quantised to E4M3(x / s) and received as
 // E4M3 * s, with binary32 division and product rounded to nearest even
-// (__fdiv_rn, __fmul_rn; the quotient as fp8_quotient gives it). Scales
-// outside [2^-125, 2^125] (whose reciprocal is not a normal number) divide
-// every value exactly.
+// (the scale as div448_rn gives it, __fmul_rn; the quotient as fp8_quotient
+// gives it). Scales outside [2^-125, 2^125] (whose reciprocal is not a normal
+// number) divide every value exactly.
 __device__ __forceinline__ void fp8_qdq8(float (&f)[8]) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-  float s = __fdiv_rn(amax, 448.0f);
+  float s = (amax >= 0x1p-120f && amax <= 0x1.fffffep127f) ? div448_rn(amax) : __fdiv_rn(amax, 448.0f);
   if (s == 0.0f) s = 1.0f;
   const bool fast = s >= 0x1p-125f && s <= 0x1p125f;
-  const float r = fast ? __frcp_rn(s) : 0.0f;
+  const float r = fast ? recip_nr(s) : 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     float lo = fast ? fp8_quotient(f[i], s, r) : __fdiv_rn(f[i], s);
