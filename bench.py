@@ -147,12 +147,31 @@ def rotation_sets(set_bytes: int, l2_bytes: int = L2_BYTES, cap: int = 64) -> in
 
 
 def load_peaks(path: str = os.path.join(ROOT, "MEASURED_PEAKS.json")):
+    """The measured HBM copy bandwidth (GB/s): the first numeric "hbm_gbs" in
+    the file, at the top level or nested; else the fallback."""
+    def find(d):
+        if isinstance(d, dict):
+            v = d.get("hbm_gbs")
+            if isinstance(v, (int, float)) and v > 0:
+                return float(v)
+            for x in d.values():
+                r = find(x)
+                if r:
+                    return r
+        elif isinstance(d, list):
+            for x in d:
+                r = find(x)
+                if r:
+                    return r
+        return None
     try:
         with open(path) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+            v = find(json.load(f))
+        if v:
+            return v, "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        pass
+    return FALLBACK_HBM_GBS, "fallback"
 
 
 def parse_clocks_csv(text: str):

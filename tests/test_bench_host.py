@@ -1,6 +1,7 @@
 """Host logic of bench.py on the CPU: bandwidth arithmetic, buffer rotation,
 clock parsing, and the multi-rank timing reduction on 2 gloo ranks."""
 
+import json
 import os
 import socket
 
@@ -66,6 +67,12 @@ def test_peaks_fallback(tmp_path):
     p = tmp_path / "p.json"
     p.write_text('{"hbm_gbs": 6451.5}')
     assert bench.load_peaks(str(p)) == (6451.5, "measured")
+    nested = tmp_path / "nested.json"
+    nested.write_text(json.dumps({"gpu": "B200", "peaks": {"hbm_gbs": 6400.0, "bf16_tflops": 1590.0}}))
+    assert bench.load_peaks(str(nested)) == (6400.0, "measured")
+    junk = tmp_path / "junk.json"
+    junk.write_text(json.dumps({"hbm_gbs": "fast"}))
+    assert bench.load_peaks(str(junk)) == (bench.FALLBACK_HBM_GBS, "fallback")
 
 
 def _free_port():
