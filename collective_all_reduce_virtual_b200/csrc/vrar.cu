@@ -487,6 +487,12 @@ constexpr int kPullThreads = 256;
 // against 2.51 us).
 constexpr size_t kPlainTwoPerSmBytes = 32u << 20;
 
+// Above that size the one-CTA build runs on at most this many CTAs: fewer
+// concurrent streams draw more from DRAM (at 8 x 224 MiB: 608.5 against 620.4
+// us with 144 CTAs; 16 x 64 MiB: 343.1 against 348.9; 16 x 32 MiB: 171.7
+// against 174.5; 112 CTAs are slower again: 643.8 us at 8 x 224 MiB).
+constexpr int kPlainDramCtas = 128;
+
 // Kernels of the custom all-reduce (one-shot, pull 2-stage, plain write), with
 // or without the fp8 wire (q8, 16-bit element types only; the host rejects
 // fp8 for fp32 before it gets here). two_per_sm picks the plain write kernel's
@@ -921,10 +927,13 @@ int vrar_allreduce(const void* const rank_in[], void* const rank_out[], int P, s
   if (algo == VRAR_ALGO_TWOSTAGE) threads = kPullThreads;
   fn = custom_kernel_dt(dtype, algo, threads, q8);
   int budget = grid_budget(fn, dev, sms, threads);
-  if (algo == VRAR_ALGO_TWOSTAGE_WRITE && !q8 && 2 * static_cast<size_t>(P) * n * elem_size(dtype) <= kPlainTwoPerSmBytes &&
+  const size_t call_bytes = 2 * static_cast<size_t>(P) * n * elem_size(dtype);
+  if (algo == VRAR_ALGO_TWOSTAGE_WRITE && !q8 && call_bytes <= kPlainTwoPerSmBytes &&
       work > static_cast<int64_t>(std::min(budget, kMaxCtas) / P) * threads) {
     fn = custom_kernel_dt(dtype, algo, threads, false, true);  // one pass needs two CTAs per SM
     budget = grid_budget(fn, dev, sms, threads);
+  } else if (algo == VRAR_ALGO_TWOSTAGE_WRITE && !q8 && call_bytes > kPlainTwoPerSmBytes) {
+    budget = std::min(budget, kPlainDramCtas);
   }
   a.B = blocks_per_rank(work, P, budget, threads);
   return launch(fn, a, a.B * P, reinterpret_cast<cudaStream_t>(stream), threads);
