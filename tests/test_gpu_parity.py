@@ -528,12 +528,13 @@ def test_payload_slots_are_bounded_by_the_grid():
     one_round = lambda P, items, steps: P * steps * items * 32  # noqa: E731
     # 8 x 128 KiB: one round, one slot per item
     assert vrar.workspace_bytes(8, 65_536, torch.bfloat16, "rd") == one_round(8, 8192, 3)
+    # several rounds: two slot sets of at most one resident grid's slots, whatever the message
+    # (rounds are evened out, so the grid, and with it the slots, may shrink a little)
     big = [vrar.workspace_bytes(8, n, torch.bfloat16, "rd") for n in (1 << 22, 1 << 24, 16384 * 7168)]
-    assert big[0] == big[1] == big[2], big
+    assert max(big) <= 64 << 20 and min(big) >= max(big) // 2, big
     assert big[2] < one_round(8, (16384 * 7168) // 8, 3) // 100, big
-    assert big[2] <= 64 << 20, big
     h = [vrar.workspace_bytes(32, n, torch.bfloat16, "hier") for n in (1 << 22, 1 << 24)]
-    assert h[0] == h[1] and h[1] <= 64 << 20, h
+    assert max(h) <= 64 << 20 and min(h) >= max(h) // 2, h
     # the full-size prefill through recursive doubling, against the oracle on sampled windows
     P, n = 8, 16384 * 7168
     d_in = synth.make_inputs(P, n, torch.bfloat16, synth.normal(0.0, 0.02), seed=0, device="cuda", block=1 << 25)
