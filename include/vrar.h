@@ -233,8 +233,10 @@ VRAR_API int vrar_get_fp8_quant(void);
 VRAR_API int vrar_set_edge_sync(int on);
 VRAR_API int vrar_get_edge_sync(void);
 
-/* Upper bound on the CTAs one call launches (default 0 = as many as fit on
- * the device at once; every call still gets at least one CTA per rank). A
+/* Upper bound on the CTAs one call launches (default 0 = the library's own
+ * choice, at most what fits on the device at once: e.g. the plain write
+ * kernel takes at most 128 on calls above 32 MiB, and recursive doubling
+ * evens out its rounds; every call still gets at least one CTA per rank). A
  * budget leaves SMs to work running concurrently on other streams, e.g. the
  * partner micro-batch's GEMMs while this all-reduce runs on a communication
  * stream; the all-reduce is bound by memory bandwidth, which a fraction of
